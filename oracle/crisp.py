@@ -1,0 +1,409 @@
+"""Float64 CPU restatement of CRISP sparse prefill (test infrastructure only).
+
+Notation follows the CRISP paper: n keys, head dim d, block size B,
+N_b = n / B blocks, representative query block Q_hat = the last b = B query
+rows, proxy map A_hat = Softmax(Q_hat K^T / sqrt(d)).
+
+Readings of steps the paper leaves open (each is stated where it is used):
+  * A_hat is causal (query row r sits at position n - b + r).
+  * blockpool sums the per-key means inside a block, so the block scores of
+    each direction sum to one (the only reading under which Eq. 3's
+    "1 - p[0] - p[N_b-1]" is a residual mass).
+  * the slash (diagonal) index of entry (r, j) is j + (b - 1 - r), the key
+    where its diagonal meets the last query row; so slash block 0 is the
+    farthest diagonals and slash block N_b-1 the local ones.
+  * decisions (route, threshold compare, top-k, gamma cut) are taken on
+    float32 values, the kernel's precision; the scores feeding them are
+    computed in float64 and rounded once.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+__all__ = [
+    "VS", "PE", "CrispParams", "bf16_to_f64", "proxy_attention", "vertical_slash_scores",
+    "c_struct_from_map", "route_cstruct", "pooled_estimate_last_block", "js_distance",
+    "route_jsd", "noise_floor", "vs_index_alpha", "vs_index_gamma", "pe_pool",
+    "pe_estimate", "pe_index", "vs_tile_mask", "vs_tile_mask_tokenwise", "pe_tile_mask",
+    "masked_attention_rows", "head_route_and_select", "crisp_prefill",
+]
+
+VS, PE = 0, 1
+
+
+@dataclass
+class CrispParams:
+    """Hyper-parameters of one CRISP prefill (CRISP paper, Section 5 Setup)."""
+
+    block: int = 128
+    alpha: float = 1.0
+    gamma: float = 0.95
+    tau_proxy: float = 0.2
+    tau_jsd: float = 0.1
+    k_min_blocks: int = 8
+    router: str = "cstruct"   # "cstruct" (Eq. 2) or "jsd" (Appendix A, Algorithm 5)
+    vs_rule: str = "alpha"    # "alpha" (Algorithm 3) or "gamma" (Appendix A, Algorithm 6)
+    sm_scale: float = 0.0     # 0 -> 1/sqrt(d)
+
+    def scale(self, d: int) -> float:
+        return self.sm_scale if self.sm_scale > 0 else 1.0 / math.sqrt(d)
+
+
+def bf16_to_f64(t) -> np.ndarray:
+    """Exact widening of a torch bfloat16 tensor to a float64 numpy array."""
+    import torch
+    return t.detach().to("cpu").to(torch.float32).numpy().astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# (a) Proxy attention — CRISP paper, Algorithm 2 (PatSearch), lines 3-5.
+# ---------------------------------------------------------------------------
+def proxy_attention(q_hat: np.ndarray, k: np.ndarray, scale: float) -> np.ndarray:
+    """A_hat = Softmax(Q_hat K^T * scale) with causal masking.
+
+    q_hat: [b, d] — the last b query rows (Algorithm 2, line 3).
+    k:     [n, d] — all keys.  Row r of q_hat is at position n - b + r and
+    sees keys j <= n - b + r (reading: causal prefill).
+    Returns [b, n] float64; masked entries are exactly 0.
+    """
+    b, n = q_hat.shape[0], k.shape[0]
+    logits = (q_hat @ k.T) * scale
+    pos = n - b + np.arange(b)
+    visible = np.arange(n)[None, :] <= pos[:, None]
+    logits = np.where(visible, logits, -np.inf)
+    m = logits.max(axis=1, keepdims=True)
+    e = np.exp(logits - m)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def vertical_slash_scores(a_hat: np.ndarray, block: int):
+    """Block scores p_v, p_s of Algorithm 3, lines 3-5.
+
+    a_v = colmean(A_hat): mean over the b proxy rows of each key column.
+    a_s = diagmean(A_hat): mean over rows of the entries on each diagonal,
+    the diagonal of entry (r, j) indexed by j + (b - 1 - r).
+    blockpool: sum of the per-key (per-diagonal) means inside each block.
+    """
+    b, n = a_hat.shape
+    nb = n // block
+    a_v = a_hat.mean(axis=0)
+    a_s = np.zeros(n)
+    for r in range(b):
+        shift = b - 1 - r
+        a_s[shift:] += a_hat[r, : n - shift]
+    a_s /= b
+    return a_v.reshape(nb, block).sum(axis=1), a_s.reshape(nb, block).sum(axis=1)
+
+
+def c_struct_from_map(a_hat: np.ndarray, block: int) -> float:
+    """Eq. 2: mean over proxy rows of the mass at the anchor positions.
+
+    Anchors: the sink window (first block) and the local recency window
+    (last block); Section 4.3 states these windows are exactly the first and
+    last block (reading at B=64: one block, not 128 tokens).
+    """
+    b, n = a_hat.shape
+    anchors = np.zeros(n, dtype=bool)
+    anchors[:block] = True
+    anchors[n - block:] = True
+    return float(a_hat[:, anchors].sum() / b)
+
+
+def route_cstruct(c: float, tau: float) -> int:
+    """Algorithm 2, lines 9-13: VS iff C_struct >= tau_proxy (float32 compare)."""
+    return VS if np.float32(c) >= np.float32(tau) else PE
+
+
+# ---------------------------------------------------------------------------
+# JSD router (comparison path) — CRISP paper, Appendix A, Algorithm 5.
+# ---------------------------------------------------------------------------
+def pooled_estimate_last_block(q_hat: np.ndarray, k: np.ndarray, block: int, scale: float):
+    """a_bar = Softmax(pool(Q_hat) pool(K)^T * scale) over all key blocks (line 3).
+
+    pool = block mean. The last query block sees every key block, so no
+    block-level causal mask applies.
+    """
+    n, d = k.shape
+    k_bar = k.reshape(n // block, block, d).mean(axis=1)
+    q_bar = q_hat.mean(axis=0)
+    z = (k_bar @ q_bar) * scale
+    z = z - z.max()
+    e = np.exp(z)
+    return e / e.sum()
+
+
+def _kl(p: np.ndarray, m: np.ndarray) -> float:
+    nz = p > 0
+    return float(np.sum(p[nz] * np.log(p[nz] / m[nz])))
+
+
+def js_distance(a_hat: np.ndarray, a_bar: np.ndarray) -> float:
+    """Algorithm 5, line 5: D_JS = sqrt(KL(a_hat||m)/2 + KL(a_bar||m)/2), m = mean.
+
+    Natural logarithm; 0*log(0) = 0.
+    """
+    m = 0.5 * (a_hat + a_bar)
+    return math.sqrt(max(0.5 * _kl(a_hat, m) + 0.5 * _kl(a_bar, m), 0.0))
+
+
+def route_jsd(djs: float, tau: float) -> int:
+    """Algorithm 5, lines 6-10: VS iff D_JS >= tau (float32 compare)."""
+    return VS if np.float32(djs) >= np.float32(tau) else PE
+
+
+# ---------------------------------------------------------------------------
+# (b) Sink-aware vertical-slash selection — Algorithm 3, Eq. 3 and Eq. 4.
+# ---------------------------------------------------------------------------
+def noise_floor(p: np.ndarray) -> np.float32:
+    """Eq. 3 / Algorithm 3 lines 7-8: mu = max(1 - p[0] - p[N_b-1], 0) / (N_b - 2)."""
+    p32 = p.astype(np.float32)
+    nb = p32.shape[0]
+    r = np.float32(1.0) - p32[0] - p32[nb - 1]
+    r = max(r, np.float32(0.0))
+    return np.float32(r / np.float32(nb - 2))
+
+
+def _topk_desc(values32: np.ndarray, k: int) -> np.ndarray:
+    """Indices of the k largest values; equal values -> lower index first."""
+    order = np.lexsort((np.arange(values32.shape[0]), -values32.astype(np.float64)))
+    return np.sort(order[:k])
+
+
+def vs_index_alpha(p: np.ndarray, alpha: float, k_min: int) -> np.ndarray:
+    """Algorithm 3, lines 7-12 for one direction.
+
+    k_d = #{j : p[j] > alpha * mu} over all blocks (Eq. 4, strict),
+    clipped to [k_min, N_b]; S_d = top-k_d(p). Returns sorted block ids.
+    """
+    p32 = p.astype(np.float32)
+    nb = p32.shape[0]
+    thr = np.float32(np.float32(alpha) * noise_floor(p))
+    k = int(np.count_nonzero(p32 > thr))
+    k = min(max(k, k_min), nb)
+    return _topk_desc(p32, k)
+
+
+def _gamma_count(sorted_desc32: np.ndarray, gamma: float) -> int:
+    """Smallest k with sum of the first k sorted values >= gamma, else all."""
+    cs = np.cumsum(sorted_desc32.astype(np.float64))
+    hit = np.nonzero(cs >= np.float64(np.float32(gamma)))[0]
+    return int(hit[0]) + 1 if hit.size else int(sorted_desc32.shape[0])
+
+
+def vs_index_gamma(p: np.ndarray, gamma: float, k_min: int) -> np.ndarray:
+    """Appendix A, Algorithm 6, one direction: sort descending, accumulate to gamma.
+
+    p is already normalised (Algorithm 6 lines 2-3 divide by the total mass,
+    which p_v / p_s carry as 1). Reading: the same k_min floor as
+    Algorithm 3, so the two rules differ only in the budget.
+    """
+    p32 = p.astype(np.float32)
+    nb = p32.shape[0]
+    order = np.lexsort((np.arange(nb), -p32.astype(np.float64)))
+    k = _gamma_count(p32[order], gamma)
+    k = min(max(k, k_min), nb)
+    return np.sort(order[:k])
+
+
+# ---------------------------------------------------------------------------
+# (c) Pooled estimation for diffuse heads — Algorithm 4 (PE Index).
+# ---------------------------------------------------------------------------
+def pe_pool(x: np.ndarray, block: int) -> np.ndarray:
+    """Algorithm 4, line 3: block-mean pooling over all rows ([n, d] -> [N_b, d])."""
+    n, d = x.shape
+    return x.reshape(n // block, block, d).mean(axis=1)
+
+
+def pe_estimate(q_bar: np.ndarray, k_bar: np.ndarray, scale: float) -> np.ndarray:
+    """Algorithm 4, line 4: A_bar = Softmax(Q_bar K_bar^T * scale).
+
+    Reading: causal at block level (query block i sees key blocks j <= i).
+    Returns [N_b, N_b]; entries above the diagonal are 0.
+    """
+    nb = q_bar.shape[0]
+    z = (q_bar @ k_bar.T) * scale
+    z = np.where(np.tril(np.ones((nb, nb), dtype=bool)), z, -np.inf)
+    z = z - z.max(axis=1, keepdims=True)
+    e = np.exp(z)
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def pe_index(a_bar: np.ndarray, gamma: float) -> np.ndarray:
+    """Algorithm 4, lines 6-10: normalise, flatten, sort descending, gamma-cumsum.
+
+    Flattening covers the causal (lower-triangle) entries in row-major order;
+    flat id = i * N_b + j. Equal values -> lower flat id first.
+    Returns the selected flat ids (unsorted = selection order).
+    """
+    nb = a_bar.shape[0]
+    ii, jj = np.tril_indices(nb)
+    total = a_bar[ii, jj].sum()
+    vals32 = (a_bar[ii, jj] / total).astype(np.float32)
+    flat = ii.astype(np.int64) * nb + jj
+    order = np.lexsort((flat, -vals32.astype(np.float64)))
+    k = _gamma_count(vals32[order], gamma)
+    return flat[order[:k]]
+
+
+# ---------------------------------------------------------------------------
+# (d) Tile masks and masked attention — Eq. 1.
+# ---------------------------------------------------------------------------
+def vs_tile_mask(s_v: Sequence[int], s_s: Sequence[int], nb: int) -> np.ndarray:
+    """Tile (qb, kb) of a VS head is computed iff it holds a selected entry.
+
+    Algorithm 3 returns S_v U S_s U {0, N_b-1}: vertical block ids and slash
+    block ids, plus the always-kept first and last block (read as vertical
+    block 0 and slash block N_b-1; every reading gives the same tiles).
+    Slash block jb covers key-query offsets [ob*B, ob*B + B - 1] with
+    ob = N_b - 1 - jb, which meet tile (qb, kb) exactly when qb - kb is ob or
+    ob + 1. Tiles are computed whole (plus the causal mask in-tile).
+    """
+    mask = np.zeros((nb, nb), dtype=bool)
+    cols = set(int(x) for x in s_v) | {0}
+    offs = set(nb - 1 - int(x) for x in s_s) | {0}
+    for qb in range(nb):
+        for kb in range(qb + 1):
+            dlt = qb - kb
+            if kb in cols or dlt in offs or (dlt - 1) in offs:
+                mask[qb, kb] = True
+    return mask
+
+
+def vs_tile_mask_tokenwise(s_v, s_s, n: int, block: int) -> np.ndarray:
+    """Brute-force definition of the same tile mask, token by token.
+
+    Query t attends key j <= t iff block(j) is a selected vertical block, or
+    the slash index n - 1 - (t - j) falls in a selected slash block (with
+    vertical 0 and slash N_b-1 always kept). A tile is computed iff any of
+    its (t, j) pairs is kept. O(n^2): small n only.
+    """
+    nb = n // block
+    cols = set(int(x) for x in s_v) | {0}
+    slash = set(int(x) for x in s_s) | {nb - 1}
+    mask = np.zeros((nb, nb), dtype=bool)
+    for t in range(n):
+        for j in range(t + 1):
+            if (j // block) in cols or ((n - 1 - (t - j)) // block) in slash:
+                mask[t // block, j // block] = True
+    return mask
+
+
+def pe_tile_mask(selected_flat: np.ndarray, nb: int) -> np.ndarray:
+    """PE tile mask: the Algorithm 4 selection plus, for every query block,
+    its diagonal tile and key block 0 (reading: keeps every query row's
+    softmax defined; consistent with the always-retained first/last blocks
+    of Section 4.3)."""
+    mask = np.zeros((nb, nb), dtype=bool)
+    mask.flat[np.asarray(selected_flat, dtype=np.int64)] = True
+    idx = np.arange(nb)
+    mask[idx, idx] = True
+    mask[:, 0] = True
+    return mask
+
+
+def masked_attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, tile_mask: np.ndarray,
+                          block: int, scale: float, qblocks: Optional[Sequence[int]] = None):
+    """Eq. 1: O = Softmax(Q K^T * scale + M_S) V with M_S from whole tiles
+    and the causal mask; float64 throughout.
+
+    Returns (O [len(rows), d], lse [len(rows)], rows) for the listed query
+    blocks (all when None). lse is the natural-log sum of exp of the logits.
+    """
+    n, d = q.shape
+    nb = n // block
+    qbs = list(range(nb)) if qblocks is None else list(qblocks)
+    outs, lses, rows = [], [], []
+    for qb in qbs:
+        kbs = np.nonzero(tile_mask[qb, : qb + 1])[0]
+        keys = (kbs[:, None] * block + np.arange(block)[None, :]).reshape(-1)
+        t = qb * block + np.arange(block)
+        z = (q[t] @ k[keys].T) * scale
+        z = np.where(keys[None, :] <= t[:, None], z, -np.inf)
+        m = z.max(axis=1, keepdims=True)
+        e = np.exp(z - m)
+        s = e.sum(axis=1, keepdims=True)
+        outs.append((e @ v[keys]) / s)
+        lses.append((m + np.log(s))[:, 0])
+        rows.append(t)
+    return np.concatenate(outs), np.concatenate(lses), np.concatenate(rows)
+
+
+# ---------------------------------------------------------------------------
+# Algorithm 1 per head, and the whole prefill.
+# ---------------------------------------------------------------------------
+def head_route_and_select(q_head: np.ndarray, k_head: np.ndarray, prm: CrispParams,
+                          force_pattern: Optional[int] = None) -> Dict[str, object]:
+    """Algorithm 1 for one query head: PatSearch, then VSIndex or PEIndex.
+
+    q_head, k_head: float64 [n, d]. ``force_pattern`` overrides the route
+    (used to compare later stages on the GPU's route for exempt heads).
+    """
+    n, d = q_head.shape
+    B = prm.block
+    nb = n // B
+    scale = prm.scale(d)
+    q_hat = q_head[n - B:]
+    a_hat = proxy_attention(q_hat, k_head, scale)
+    p_v, p_s = vertical_slash_scores(a_hat, B)
+    c = c_struct_from_map(a_hat, B)
+    out: Dict[str, object] = {"p_v": p_v, "p_s": p_s, "c_struct": c}
+    if prm.router == "jsd":
+        a_bar = pooled_estimate_last_block(q_hat, k_head, B, scale)
+        djs = js_distance(p_v, a_bar)
+        out["d_js"] = djs
+        pattern = route_jsd(djs, prm.tau_jsd)
+        out["score"] = djs
+    else:
+        pattern = route_cstruct(c, prm.tau_proxy)
+        out["score"] = c
+    out["routed"] = pattern
+    if force_pattern is not None:
+        pattern = force_pattern
+    out["pattern"] = pattern
+    if pattern == VS:
+        if prm.vs_rule == "gamma":
+            s_v = vs_index_gamma(p_v, prm.gamma, prm.k_min_blocks)
+            s_s = vs_index_gamma(p_s, prm.gamma, prm.k_min_blocks)
+        else:
+            s_v = vs_index_alpha(p_v, prm.alpha, prm.k_min_blocks)
+            s_s = vs_index_alpha(p_s, prm.alpha, prm.k_min_blocks)
+        out["s_v"], out["s_s"] = s_v, s_s
+        out["mask"] = vs_tile_mask(s_v, s_s, nb)
+    else:
+        a_bar = pe_estimate(pe_pool(q_head, B), pe_pool(k_head, B), scale)
+        sel = pe_index(a_bar, prm.gamma)
+        out["a_bar"] = a_bar
+        out["pe_selected"] = sel
+        out["mask"] = pe_tile_mask(sel, nb)
+    return out
+
+
+def crisp_prefill(q, k, v, prm: CrispParams, qblocks: Optional[Sequence[int]] = None,
+                  heads: Optional[Sequence[int]] = None, force_patterns: Optional[dict] = None,
+                  masks: Optional[dict] = None) -> Dict[str, object]:
+    """Algorithm 1 over a whole [batch, H, n, d] problem (float64 numpy inputs).
+
+    GQA: query head h reads KV head h // (H_q / H_kv). ``masks`` (keyed by
+    (batch, head)) replaces the oracle's own tile masks for the attention
+    step, so attention can be compared on another implementation's mask.
+    Returns per (batch, head) dicts under "heads" and attention rows.
+    """
+    bsz, hq, n, d = q.shape
+    hkv = k.shape[1]
+    g = hq // hkv
+    scale = prm.scale(d)
+    res: Dict[str, object] = {"heads": {}, "attn": {}}
+    heads = list(range(hq)) if heads is None else list(heads)
+    for b in range(bsz):
+        for h in heads:
+            fp = None if force_patterns is None else force_patterns.get((b, h))
+            hr = head_route_and_select(q[b, h], k[b, h // g], prm, force_pattern=fp)
+            res["heads"][(b, h)] = hr
+            mask = hr["mask"] if masks is None else masks[(b, h)]
+            res["attn"][(b, h)] = masked_attention_rows(q[b, h], k[b, h // g], v[b, h // g],
+                                                        mask, prm.block, scale, qblocks)
+    return res

@@ -1,0 +1,396 @@
+"""Pins of the CPU oracle against facts it does not compute itself.
+
+Each test checks one oracle function against brute force written a second
+way, a closed form from the CRISP paper (Appendix C), a hand-computed case
+(tests/golden), an invariant, or planted-structure recovery.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+# --------------------------------------------------------------------------- proxy map
+def _proxy_bruteforce(q_hat, k, scale):
+    b, n = len(q_hat), len(k)
+    out = [[0.0] * n for _ in range(b)]
+    for r in range(b):
+        t = n - b + r
+        logits = []
+        for j in range(t + 1):
+            logits.append(sum(q_hat[r][c] * k[j][c] for c in range(len(k[j]))) * scale)
+        mx = max(logits)
+        den = sum(math.exp(z - mx) for z in logits)
+        for j in range(t + 1):
+            out[r][j] = math.exp(logits[j] - mx) / den
+    return np.array(out)
+
+
+def test_proxy_matches_bruteforce():
+    rng = _rng(1)
+    q_hat = rng.standard_normal((4, 8))
+    k = rng.standard_normal((24, 8))
+    got = O.proxy_attention(q_hat, k, 0.7)
+    want = _proxy_bruteforce(q_hat.tolist(), k.tolist(), 0.7)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-13)
+
+
+def test_proxy_rows_sum_to_one_and_causal_zeros():
+    rng = _rng(2)
+    q_hat = rng.standard_normal((16, 8))
+    k = rng.standard_normal((64, 8))
+    a = O.proxy_attention(q_hat, k, 0.3)
+    np.testing.assert_allclose(a.sum(axis=1), 1.0, atol=1e-14)
+    for r in range(16):
+        assert np.all(a[r, 64 - 16 + r + 1:] == 0.0)
+        assert np.all(a[r, : 64 - 16 + r + 1] > 0.0)
+
+
+def test_appendix_c_background_mass_closed_form():
+    """App. C: k signal keys at logit z, n-k background keys at z - Delta give each
+    background key mass e^-D / (k + (n-k) e^-D); n = keys visible to the row."""
+    n, b, d = 96, 8, 4
+    z, delta, sig = 3.0, 2.5, [0, 1, 2, 3, 40, 41]
+    q_hat = np.zeros((b, d))
+    q_hat[:, 0] = 1.0
+    k = np.zeros((n, d))
+    k[:, 0] = z - delta
+    k[sig, 0] = z
+    a = O.proxy_attention(q_hat, k, 1.0)
+    for r in range(b):
+        nvis = n - b + r + 1
+        eps = math.exp(-delta) / (len(sig) + (nvis - len(sig)) * math.exp(-delta))
+        bg = [j for j in range(nvis) if j not in sig]
+        np.testing.assert_allclose(a[r, bg], eps, rtol=1e-12)
+        np.testing.assert_allclose(a[r, sig], eps * math.exp(delta), rtol=1e-12)
+
+
+# --------------------------------------------------------------------------- block scores
+def test_scores_each_sum_to_one():
+    rng = _rng(3)
+    a = O.proxy_attention(rng.standard_normal((16, 8)), rng.standard_normal((128, 8)), 0.5)
+    p_v, p_s = O.vertical_slash_scores(a, 16)
+    assert p_v.shape == (8,) and p_s.shape == (8,)
+    assert abs(p_v.sum() - 1.0) < 1e-13 and abs(p_s.sum() - 1.0) < 1e-13
+
+
+def test_slash_equals_vertical_for_single_row():
+    """With one proxy row the diagonal index j + (b-1-r) is j itself."""
+    rng = _rng(4)
+    a = O.proxy_attention(rng.standard_normal((1, 8)), rng.standard_normal((64, 8)), 1.0)
+    p_v, p_s = O.vertical_slash_scores(a, 8)
+    np.testing.assert_array_equal(p_v, p_s)
+
+
+def test_slash_scores_bruteforce_diagonal_sums():
+    """diagmean written out per diagonal offset o = t - j (slash index n-1-o)."""
+    rng = _rng(5)
+    b, n, B = 8, 64, 8
+    a = O.proxy_attention(rng.standard_normal((b, 4)), rng.standard_normal((n, 4)), 1.0)
+    _, p_s = O.vertical_slash_scores(a, B)
+    want = np.zeros(n // B)
+    for r in range(b):
+        t = n - b + r
+        for j in range(t + 1):
+            o = t - j
+            want[(n - 1 - o) // B] += a[r, j] / b
+    np.testing.assert_allclose(p_s, want, atol=1e-15)
+
+
+def test_planted_exact_diagonal_goes_to_its_slash_block():
+    """K = Q shifted by delta: all proxy mass on offset delta -> one slash block."""
+    n, b, B, delta = 64, 8, 8, 19
+    d = n + delta + 1
+    q = np.zeros((n, d))
+    k = np.zeros((n, d))
+    for t in range(n):
+        q[t, t] = 30.0
+    for j in range(n):
+        k[j, j + delta] = 1.0   # q_t . k_j = 30 iff t = j + delta
+    a = O.proxy_attention(q[n - b:], k, 1.0)
+    p_v, p_s = O.vertical_slash_scores(a, B)
+    jb = (n - 1 - delta) // B
+    assert p_s[jb] > 0.999
+    # the vertical view spreads over the keys t - delta of the b rows
+    assert p_v.max() < 0.9
+
+
+# --------------------------------------------------------------------------- routing
+def test_cstruct_equals_anchor_block_scores():
+    rng = _rng(6)
+    a = O.proxy_attention(rng.standard_normal((16, 8)), rng.standard_normal((160, 8)), 0.9)
+    p_v, _ = O.vertical_slash_scores(a, 16)
+    assert abs(O.c_struct_from_map(a, 16) - (p_v[0] + p_v[-1])) < 1e-14
+
+
+def test_cstruct_uniform_head_closed_form():
+    """Q = 0: row r spreads evenly over its n-B+r+1 visible keys; anchors hold
+    the B sink keys and the r+1 visible keys of the last block."""
+    n, B, d = 512, 32, 8
+    q_hat = np.zeros((B, d))
+    k = _rng(7).standard_normal((n, d))
+    c = O.c_struct_from_map(O.proxy_attention(q_hat, k, 1.0), B)
+    want = np.mean([(B + r + 1) / (n - B + r + 1) for r in range(B)])
+    assert abs(c - want) < 1e-14
+    assert O.route_cstruct(c, 0.2) == O.PE
+
+
+def test_route_threshold_is_inclusive():
+    assert O.route_cstruct(0.2, 0.2) == O.VS
+    assert O.route_cstruct(np.nextafter(np.float32(0.2), np.float32(0)), 0.2) == O.PE
+    assert O.route_jsd(0.1, 0.1) == O.VS
+
+
+def _golden(name):
+    rows = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                key, *vals = line.split()
+                rows.setdefault(key, []).append(vals)
+    return rows
+
+
+def test_jsd_closed_forms():
+    g = _golden("jsd_closed_forms.txt")
+    a = np.array([0.2, 0.3, 0.5])
+    assert O.js_distance(a, a) == 0.0
+    d = O.js_distance(np.array([0.5, 0.5, 0, 0]), np.array([0, 0, 0.25, 0.75]))
+    assert abs(d - float(g["disjoint"][0][0])) < 1e-15
+    assert abs(d - math.sqrt(math.log(2))) < 1e-15
+    h = O.js_distance(np.array([1.0, 0.0]), np.array([0.5, 0.5]))
+    assert abs(h - float(g["half"][0][0])) < 1e-15
+
+
+def test_jsd_symmetric_and_bounded():
+    rng = _rng(8)
+    for _ in range(20):
+        x = rng.random(12) ** 3
+        y = rng.random(12) ** 3
+        x /= x.sum()
+        y /= y.sum()
+        d1, d2 = O.js_distance(x, y), O.js_distance(y, x)
+        assert abs(d1 - d2) < 1e-15
+        assert 0.0 <= d1 <= math.sqrt(math.log(2)) + 1e-15
+
+
+def test_pooled_estimate_bruteforce():
+    rng = _rng(9)
+    q_hat = rng.standard_normal((4, 3))
+    k = rng.standard_normal((12, 3))
+    got = O.pooled_estimate_last_block(q_hat, k, 4, 0.5)
+    qm = [sum(q_hat[r][c] for r in range(4)) / 4 for c in range(3)]
+    z = []
+    for kb in range(3):
+        km = [sum(k[kb * 4 + i][c] for i in range(4)) / 4 for c in range(3)]
+        z.append(0.5 * sum(qm[c] * km[c] for c in range(3)))
+    e = [math.exp(x) for x in z]
+    np.testing.assert_allclose(got, [x / sum(e) for x in e], atol=1e-15)
+
+
+# --------------------------------------------------------------------------- selection
+def test_alpha_rule_hand_cases():
+    g = _golden("alpha_rule_hand.txt")
+    p = np.array([float(x) for x in g["p"][0]])
+    for vals in g["case"]:
+        alpha = float(vals[0].split("=")[1])
+        kmin = int(vals[1].split("=")[1])
+        want = [int(x) for x in vals[3:]]
+        got = O.vs_index_alpha(p, alpha, kmin)
+        assert got.tolist() == want, (alpha, kmin, got)
+    assert abs(float(O.noise_floor(p)) - 0.0425) < 1e-8
+
+
+def test_noise_floor_clamps_at_zero():
+    p = np.array([0.7, 0.0, 0.0, 0.4])   # first + last > 1
+    assert float(O.noise_floor(p)) == 0.0
+    # every block with positive score passes a zero floor
+    assert O.vs_index_alpha(p, 1.0, 1).tolist() == [0, 3]
+
+
+def test_alpha_rule_clips_to_nb():
+    p = np.full(6, 1 / 6)
+    assert O.vs_index_alpha(p, 0.5, 8).tolist() == list(range(6))
+
+
+def _failure_vectors():
+    nb = 32
+    col = np.full(nb, 0.02 / 30)
+    col[0], col[7] = 0.96, 0.02
+    acc = np.full(nb, 0.295 / 30)
+    acc[0], acc[5] = 0.505, 0.2
+    return col, acc
+
+
+def test_gamma_sink_only_collapse_and_noise_accumulation():
+    g = _golden("gamma_failure_modes.txt")
+    col, acc = _failure_vectors()
+    assert len(O.vs_index_gamma(col, 0.95, 1)) == int(g["collapse_gamma_k"][0][0])
+    assert 7 not in O.vs_index_gamma(col, 0.95, 1)
+    sel = O.vs_index_alpha(col, 1.0, 1)
+    assert len(sel) == int(g["collapse_alpha_k"][0][0]) and 7 in sel
+    assert len(O.vs_index_gamma(acc, 0.95, 1)) == int(g["accumulate_gamma_k"][0][0])
+    assert O.vs_index_alpha(acc, 1.0, 1).tolist() == [0, 5]
+    assert len(O.vs_index_alpha(acc, 1.0, 1)) == int(g["accumulate_alpha_k"][0][0])
+
+
+def test_gamma_noise_count_grows_linearly_with_nb():
+    """App. C: the gamma cut collects ~ gamma_residual * n background blocks."""
+    counts = []
+    for nb in (64, 128, 256, 512):
+        p = np.full(nb, 0.3 / (nb - 2))
+        p[0], p[1] = 0.5, 0.2
+        counts.append(len(O.vs_index_gamma(p, 0.95, 1)) - 2)
+        assert len(O.vs_index_alpha(p, 1.0, 1)) == 2
+    for nb, c in zip((64, 128, 256, 512), counts):
+        assert abs(c - (0.25 / 0.3) * (nb - 2)) <= 1.0
+
+
+def test_gamma_takes_all_when_total_short():
+    p = np.full(10, 0.09)   # total 0.9 < gamma
+    assert len(O.vs_index_gamma(p, 0.95, 1)) == 10
+
+
+def test_gamma_ties_break_to_lower_index():
+    p = np.array([0.4, 0.2, 0.2, 0.2])
+    assert O.vs_index_gamma(p, 0.75, 1).tolist() == [0, 1, 2]
+
+
+def test_pe_pool_and_estimate_bruteforce():
+    rng = _rng(10)
+    x = rng.standard_normal((12, 3))
+    pooled = O.pe_pool(x, 4)
+    for i in range(3):
+        np.testing.assert_allclose(pooled[i], x[4 * i:4 * i + 4].sum(axis=0) / 4, atol=1e-15)
+    qb, kb = rng.standard_normal((4, 3)), rng.standard_normal((4, 3))
+    a = O.pe_estimate(qb, kb, 0.3)
+    for i in range(4):
+        z = [0.3 * float(qb[i] @ kb[j]) for j in range(i + 1)]
+        e = [math.exp(v) for v in z]
+        np.testing.assert_allclose(a[i, : i + 1], [v / sum(e) for v in e], atol=1e-15)
+        assert np.all(a[i, i + 1:] == 0)
+
+
+def test_pe_index_hand_case():
+    # rows: [1], [0.7, 0.3], [0.5, 0.3, 0.2]; total 3 -> normalised /3
+    a = np.array([[1.0, 0, 0], [0.7, 0.3, 0], [0.5, 0.3, 0.2]])
+    # sorted: 1/3 (0,0), 0.7/3 (1,0), 0.5/3 (2,0), 0.3/3 (1,1), 0.3/3 (2,1), 0.2/3 (2,2)
+    sel = O.pe_index(a, 0.8)    # cumsum 1/3, 1.7/3, 2.2/3, 2.5/3 >= 0.8 -> 4 entries
+    assert sel.tolist() == [0, 3, 6, 4]
+    m = O.pe_tile_mask(sel, 3)
+    assert m.tolist() == [[1, 0, 0], [1, 1, 0], [1, 0, 1]]
+
+
+def test_vs_tile_mask_matches_tokenwise_definition():
+    rng = _rng(11)
+    for trial in range(12):
+        B, nb = 4, int(rng.integers(3, 12))
+        n = nb * B
+        s_v = rng.choice(nb, size=int(rng.integers(0, nb)), replace=False)
+        s_s = rng.choice(nb, size=int(rng.integers(0, nb)), replace=False)
+        a = O.vs_tile_mask(s_v, s_s, nb)
+        b = O.vs_tile_mask_tokenwise(s_v, s_s, n, B)
+        np.testing.assert_array_equal(a, b)
+
+
+# --------------------------------------------------------------------------- attention
+def _attention_bruteforce(q, k, v, allowed, scale):
+    n, d = len(q), len(q[0])
+    out, lse = [], []
+    for t in range(n):
+        z = [(j, sum(q[t][c] * k[j][c] for c in range(d)) * scale) for j in range(n) if allowed(t, j)]
+        mx = max(x for _, x in z)
+        w = [(j, math.exp(x - mx)) for j, x in z]
+        s = sum(x for _, x in w)
+        out.append([sum(x * v[j][c] for j, x in w) / s for c in range(d)])
+        lse.append(mx + math.log(s))
+    return np.array(out), np.array(lse)
+
+
+def test_masked_attention_bruteforce():
+    rng = _rng(12)
+    n, d, B = 32, 4, 8
+    q, k, v = rng.standard_normal((3, n, d))
+    mask = rng.random((4, 4)) < 0.5
+    np.fill_diagonal(mask, True)
+    o, lse, rows = O.masked_attention_rows(q, k, v, mask, B, 0.6)
+    want_o, want_lse = _attention_bruteforce(q.tolist(), k.tolist(), v.tolist(),
+                                             lambda t, j: j <= t and mask[t // B, j // B], 0.6)
+    np.testing.assert_allclose(o, want_o, atol=1e-13)
+    np.testing.assert_allclose(lse, want_lse, atol=1e-13)
+    assert rows.tolist() == list(range(n))
+
+
+def test_full_mask_equals_dense_causal_softmax():
+    rng = _rng(13)
+    n, d, B = 48, 6, 8
+    q, k, v = rng.standard_normal((3, n, d))
+    full = np.tril(np.ones((6, 6), dtype=bool))
+    o, _, _ = O.masked_attention_rows(q, k, v, full, B, 0.4)
+    z = q @ k.T * 0.4 + np.triu(np.full((n, n), -np.inf), 1)
+    p = np.exp(z - z.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, atol=1e-14)
+    np.testing.assert_allclose(o, p @ v, atol=1e-13)
+
+
+def test_attention_is_causal():
+    rng = _rng(14)
+    n, d, B = 40, 4, 8
+    q, k, v = rng.standard_normal((3, n, d))
+    full = np.tril(np.ones((5, 5), dtype=bool))
+    o1, _, _ = O.masked_attention_rows(q, k, v, full, B, 0.5)
+    k2, v2 = k.copy(), v.copy()
+    k2[21:] += 5.0
+    v2[21:] -= 3.0
+    o2, _, _ = O.masked_attention_rows(q, k2, v2, full, B, 0.5)
+    np.testing.assert_array_equal(o1[:21], o2[:21])
+    assert not np.allclose(o1[21:], o2[21:])
+
+
+# --------------------------------------------------------------------------- planted recovery
+def test_planted_recovery_tiny_workload():
+    from synthetic import WORKLOADS, make_qkv
+    w = WORKLOADS["tiny"]
+    q, k, v, meta = make_qkv(w)
+    prm = O.CrispParams(block=w.block, alpha=1.0)
+    k0 = O.bf16_to_f64(k[0, 0])
+    h0 = O.head_route_and_select(O.bf16_to_f64(q[0, 0]), k0, prm)
+    h1 = O.head_route_and_select(O.bf16_to_f64(q[0, 1]), k0, prm)
+    assert h0["pattern"] == O.VS and h1["pattern"] == O.PE
+    assert 0 in h0["s_v"]                       # sink block
+    assert w.n_blocks - 1 in h0["s_s"]          # local diagonal block
+    assert h0["c_struct"] > 0.5 > 0.2 > h1["c_struct"]
+    assert h0["mask"].sum() < h1["mask"].sum()
+
+
+def test_planted_recovery_verticals_and_jsd_agreement():
+    from synthetic import Workload, make_qkv
+    w = Workload("small", 1, 4, 1, 128, 8192, 128, diffuse_heads=(3,))
+    q, k, v, meta = make_qkv(w)
+    kk = O.bf16_to_f64(k[0, 0])
+    vert_blocks = sorted({p // w.block for p in meta["verticals"][0]})
+    for h in range(4):
+        qq = O.bf16_to_f64(q[0, h])
+        hr = O.head_route_and_select(qq, kk, O.CrispParams(block=128))
+        hj = O.head_route_and_select(qq, kk, O.CrispParams(block=128, router="jsd"))
+        assert hr["pattern"] == hj["pattern"]
+        if h == 3:
+            assert hr["pattern"] == O.PE
+        else:
+            assert hr["pattern"] == O.VS
+            assert set(vert_blocks) <= set(hr["s_v"].tolist())
+            assert 0 in hr["s_v"].tolist()
+            # the noise floor keeps the flat background out: only the planted
+            # columns, the anchors and the k_min fill are selected
+            assert len(hr["s_v"]) <= max(8, len(vert_blocks) + 2)
