@@ -1,0 +1,404 @@
+#!/usr/bin/env python
+"""Benchmark of CRISP sparse prefill on B200 (one JSON line on rank 0).
+
+A step is one pass of the whole hot path over one synthetic input: route
+(proxy map, block scores, C_struct), select (VS / PE selection, tile lists)
+and block-sparse attention. The dense baseline (same attention kernel over
+every causal tile) is timed beside it for the speedup.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama_512k]
+  python bench.py --impl reference ...   # the CPU oracle on a bounded sample
+  python bench.py --sweep out.jsonl      # N x diffuse-fraction x alpha sweep
+
+Multi-GPU (torchrun): every rank runs its own replica (independent input,
+seed + rank); the path has no exchange step, so there is no collective on
+the data path. Timing is the max over ranks of CUDA-event time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse prefill attention ms, speedup vs own dense kernel at 128k/512k; TC util"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[3:7]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        loaded = [x for x in sm if x > 0.5 * (mx or max(sm))] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def launches_per_step(router: str) -> dict:
+    """Kernels of this library launched by one call of each stage."""
+    route = 4 + (1 if router == "jsd" else 0)      # proxy stats, merge, scores, (K pool), route
+    select = 13                                     # vs select, 2 pools, PE logits/normalise,
+    #                                                 3 x (hist, find), eq count/scan, tiles
+    return {"route": route, "select": select, "attention": 1, "total": route + select + 1}
+
+
+def executed_flops(tile_cnt_sum: int, block: int, d: int) -> float:
+    """4 * B^2 * d per executed tile (QK^T and PV); diagonal tiles count in full."""
+    return float(tile_cnt_sum) * 4.0 * block * block * d
+
+
+# ----------------------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import dynamic_block_sparse_qk_b200 as C
+    from synthetic import WORKLOADS, make_qkv
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload].with_(seed=args.seed + rank)
+    q, k, v, meta = make_qkv(w, device=str(dev))
+    p = C.params_for(q, k, block=w.block, alpha=args.alpha, gamma=args.gamma, router=args.router,
+                     vs_rule=args.vs_rule)
+    ws = C.alloc_workspace(p, dev)
+    bh, nb = p.batch * p.h_q, p.n_blocks
+    pattern = torch.empty(bh, dtype=torch.int32, device=dev)
+    score = torch.empty(bh, dtype=torch.float32, device=dev)
+    p_v = torch.empty(bh, nb, dtype=torch.float32, device=dev)
+    p_s = torch.empty(bh, nb, dtype=torch.float32, device=dev)
+    tidx = torch.empty(bh, nb, nb, dtype=torch.int32, device=dev)
+    tcnt = torch.empty(bh, nb, dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if in_bytes < 4 * L2_BYTES else None
+    stream = torch.cuda.current_stream(dev)
+
+    def step(evs=None):
+        if evs: evs[0].record(stream)
+        C.crisp_route(p, q, k, ws, pattern, score, p_v, p_s, stream=stream)
+        if evs: evs[1].record(stream)
+        C.crisp_select(p, q, k, pattern, p_v, p_s, ws, want_mask=False, tile_idx=tidx, tile_cnt=tcnt,
+                       stream=stream)
+        if evs: evs[2].record(stream)
+        C.crisp_sparse_prefill(p, q, k, v, tidx, tcnt, ws, o=o, lse=lse, stream=stream)
+        if evs: evs[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    status = C.crisp_get_device_status(ws)
+    cnt_sum = int(tcnt.sum().item())
+    n_vs = int((pattern == 0).sum().item())
+    causal_tiles = bh * nb * (nb + 1) // 2
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    per = [[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(3)] for i in range(args.steps)]
+    step_ms = [sum(x) for x in per]
+    ms_local = statistics.mean(step_ms)
+    stages = {n: statistics.mean(x[j] for x in per) for j, n in enumerate(("route", "select", "attend"))}
+
+    # dense baseline: same kernel, every causal tile (1 warm-up + args.dense_steps timed)
+    od = torch.empty_like(q)
+    C.crisp_dense_prefill(p, q, k, v, ws, o=od, lse=lse, stream=stream)
+    torch.cuda.synchronize(dev)
+    dts = []
+    for _ in range(args.dense_steps):
+        if flush is not None:
+            flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        C.crisp_dense_prefill(p, q, k, v, ws, o=od, lse=lse, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        dts.append(e0.elapsed_time(e1))
+    dense_ms = statistics.mean(dts)
+    del od
+
+    if world > 1:
+        t = torch.tensor([ms_local, dense_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms, dense_ms = float(t[0]), float(t[1])
+    else:
+        ms = ms_local
+
+    # end-to-end through the public API with host buffers (H2D inputs, D2H output)
+    e2e = None
+    if not args.no_e2e:
+        hq = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        hk = torch.empty(k.shape, dtype=k.dtype, pin_memory=True)
+        hv = torch.empty(v.shape, dtype=v.dtype, pin_memory=True)
+        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        hq.copy_(q)
+        hk.copy_(k)
+        hv.copy_(v)
+        torch.cuda.synchronize(dev)
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1) / args.steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t[0])
+        e2e = {"value": round(e2e_ms, 3), "unit": "ms",
+               "h2d_bytes_per_step": int(in_bytes), "d2h_bytes_per_step": int(o.numel() * o.element_size())}
+        del hq, hk, hv, ho
+
+    peaks = _peaks()
+    flops = executed_flops(cnt_sum, w.block, w.head_dim)
+    attn_tflops = flops / (stages["attend"] * 1e-3) / 1e12
+    dense_tflops = executed_flops(causal_tiles, w.block, w.head_dim) / (dense_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"] if stages["attend"] > 50 else peaks["bf16_tflops"]
+    line = {
+        "metric": METRIC, "value": round(ms, 3), "unit": "ms", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "h_q": w.h_q, "h_kv": w.h_kv,
+                   "head_dim": w.head_dim, "seq_len": w.seqlen, "block": w.block,
+                   "diffuse_frac": w.diffuse_frac, "alpha": args.alpha, "gamma": args.gamma,
+                   "router": args.router, "vs_rule": args.vs_rule, "parallelism": f"replicas{world}",
+                   "l2": "flushed between steps" if flush is not None else
+                         f"inputs ({in_bytes / 2**30:.1f} GiB) larger than L2"},
+        "stages_ms": {k_: round(v_, 3) for k_, v_ in stages.items()},
+        "dense_ms": round(dense_ms, 3),
+        "speedup_vs_dense": round(dense_ms / ms, 3),
+        "speedup_attend_only": round(dense_ms / stages["attend"], 3),
+        "route_select_frac": round((stages["route"] + stages["select"]) / ms, 4),
+        "density": round(cnt_sum / causal_tiles, 5), "vs_heads": n_vs, "heads": bh,
+        "executed_tiles": cnt_sum,
+        "attend_tflops": round(attn_tflops, 1), "dense_tflops": round(dense_tflops, 1),
+        "roofline": {"bound": "tensor", "kernel": "attention (sparse)", "achieved": round(attn_tflops, 1),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(attn_tflops / peak, 4),
+                     "peak_source": f"{peaks['source']} bf16 "
+                                    f"{'sustained' if peak == peaks['bf16_tflops_sustained'] else 'burst'}",
+                     "traffic": None},
+        "e2e": e2e,
+        "gpu_launches": launches_per_step(args.router)["total"] * args.steps,
+        "device_status": status,
+        "clocks": clk.summary(),
+    }
+    return line
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_inputs(w):
+    """CPU inputs of the oracle sample: one VS and one PE query head and their KV heads."""
+    from synthetic import make_qkv, head_kinds
+    diffuse = set(head_kinds(w)["diffuse"])
+    vs_head = next(h for h in range(w.h_q) if h not in diffuse)
+    pe_head = min(diffuse) if diffuse else None
+    heads = [vs_head] + ([pe_head] if pe_head is not None else [])
+    q, k, v, _ = make_qkv(w, heads_q=heads)
+    return {"q": q, "k": k, "v": v, "heads": heads, "vs_head": vs_head, "pe_head": pe_head,
+            "n_diffuse": len(diffuse)}
+
+
+def oracle_sample(w, args, inp, budget_s: float):
+    """Times the float64 oracle on a bounded sample of the workload and
+    extrapolates to one full prefill (ms). Returns (ms, description, threads)."""
+    import numpy as np
+    import oracle as O
+
+    g = w.h_q // w.h_kv
+    prm = O.CrispParams(block=w.block, alpha=args.alpha, gamma=args.gamma, router=args.router,
+                        vs_rule=args.vs_rule)
+    nb = w.n_blocks
+    sel_ms, tiles, attn_ms_per_tile = {}, {}, []
+    t_start = time.perf_counter()
+    for i, h in enumerate(inp["heads"]):
+        qh = O.bf16_to_f64(inp["q"][0, i])
+        kh = O.bf16_to_f64(inp["k"][0, h // g])
+        vh = O.bf16_to_f64(inp["v"][0, h // g])
+        t0 = time.perf_counter()
+        r = O.head_route_and_select(qh, kh, prm)
+        sel_ms[h] = (time.perf_counter() - t0) * 1e3
+        tiles[h] = int(r["mask"].sum())
+        rng = np.random.default_rng(h)
+        for qb in sorted(set([nb - 1] + [int(x) for x in rng.integers(0, nb, size=3)])):
+            if time.perf_counter() - t_start > budget_s:
+                break
+            t0 = time.perf_counter()
+            O.masked_attention_rows(qh, kh, vh, r["mask"], w.block, prm.scale(w.head_dim), [qb])
+            attn_ms_per_tile.append((time.perf_counter() - t0) * 1e3 / max(int(r["mask"][qb].sum()), 1))
+    n_pe = inp["n_diffuse"]
+    n_vs = w.h_q - n_pe
+    vs_h, pe_h = inp["vs_head"], inp["pe_head"]
+    total_sel = sel_ms[vs_h] * n_vs + (sel_ms[pe_h] * n_pe if pe_h is not None else 0.0)
+    total_tiles = tiles[vs_h] * n_vs + (tiles[pe_h] * n_pe if pe_h is not None else 0)
+    ms = total_sel + statistics.mean(attn_ms_per_tile) * total_tiles
+    desc = (f"oracle route+select timed on {len(inp['heads'])} heads (1 VS, 1 PE), attention on "
+            f"{len(attn_ms_per_tile)} sampled query blocks; extrapolated to {w.h_q} heads and "
+            f"{total_tiles} executed tiles")
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([x.get("num_threads", 1) for x in threadpool_info()] + [1])
+    except Exception:
+        threads = os.cpu_count()
+    return ms, desc, threads
+
+
+def run_reference(args):
+    from synthetic import WORKLOADS
+    w = WORKLOADS[args.workload].with_(seed=args.seed)
+    inp = oracle_inputs(w)
+    vals, desc, threads = [], "", 1
+    for i in range(args.warmup + args.steps):
+        ms, desc, threads = oracle_sample(w, args, inp, budget_s=args.cpu_budget)
+        if i >= args.warmup:
+            vals.append(ms)
+    v = statistics.mean(vals)
+    return {"metric": METRIC, "value": round(v, 1), "unit": "ms", "n_gpus": 0, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(v, 1), "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": w.name, "seq_len": w.seqlen, "h_q": w.h_q, "h_kv": w.h_kv,
+                       "head_dim": w.head_dim, "block": w.block, "alpha": args.alpha},
+            "cpu_baseline": {"value": round(v, 1), "unit": "ms", "cores": threads, "kind": "oracle",
+                             "sample": desc + " (extrapolated)"},
+            "e2e": {"value": round(v, 1), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ----------------------------------------------------------------------------- driver
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--dense-steps", type=int, default=2)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="llama_512k")
+    ap.add_argument("--alpha", type=float, default=1.0)
+    ap.add_argument("--gamma", type=float, default=0.95)
+    ap.add_argument("--router", default="cstruct")
+    ap.add_argument("--vs-rule", default="alpha")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    line = run_ours(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from synthetic import WORKLOADS
+        w = WORKLOADS[args.workload].with_(seed=args.seed)
+        ms, desc, threads = oracle_sample(w, args, oracle_inputs(w), budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(ms, 1), "unit": "ms", "cores": threads, "kind": "oracle",
+                                "sample": desc + " (extrapolated)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,16 @@
+"""B200-native CRISP sparse attention prefill (sm_100a kernels behind a C ABI).
+
+Stages (CRISP paper, Algorithm 1): crisp_route (PatSearch, Algorithm 2),
+crisp_select (Algorithms 3, 4 and 6 plus tile lists), crisp_sparse_prefill
+(block-sparse attention, Eq. 1) and crisp_dense_prefill (the same kernel
+over every causal tile).
+"""
+from .binding import (CrispError, CrispParams, PATTERN_PE, PATTERN_VS, alloc_workspace,
+                      crisp_dense_prefill, crisp_get_device_status, crisp_prefill, crisp_route,
+                      crisp_select, crisp_sparse_prefill, crisp_workspace_size, load_library,
+                      make_params, params_for)
+
+__all__ = ["CrispError", "CrispParams", "PATTERN_PE", "PATTERN_VS", "alloc_workspace",
+           "crisp_dense_prefill", "crisp_get_device_status", "crisp_prefill", "crisp_route",
+           "crisp_select", "crisp_sparse_prefill", "crisp_workspace_size", "load_library",
+           "make_params", "params_for"]

@@ -1,0 +1,213 @@
+"""ctypes binding of libcrisp.so — argument marshalling only.
+
+Every function here forwards to the C ABI declared in include/crisp.h. The
+tensors are torch CUDA tensors (PyTorch provides device memory and streams);
+all computation happens in the library's kernels. There is no fallback: if
+the library cannot be loaded, importing it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libcrisp.so")
+
+CRISP_OK = 0
+STATUS_NAMES = {0: "ok", -1: "invalid argument", -2: "unsupported shape", -3: "workspace too small",
+                -4: "CUDA error", -5: "device wait timed out", -6: "device index out of range"}
+ROUTER = {"cstruct": 0, "jsd": 1}
+VS_RULE = {"alpha": 0, "gamma": 1}
+PATTERN_VS, PATTERN_PE = 0, 1
+
+EXPORTED = ("crisp_version", "crisp_status_string", "crisp_check_params", "crisp_workspace_size",
+            "crisp_route", "crisp_select", "crisp_sparse_prefill", "crisp_dense_prefill",
+            "crisp_get_device_status")
+
+
+class CrispError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status} ({STATUS_NAMES.get(status, 'unknown')})")
+        self.status = status
+
+
+class CrispParams(ctypes.Structure):
+    """Mirror of crisp_params (include/crisp.h)."""
+
+    _fields_ = [("batch", ctypes.c_int32), ("h_q", ctypes.c_int32), ("h_kv", ctypes.c_int32),
+                ("seqlen", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("alpha", ctypes.c_float), ("gamma", ctypes.c_float), ("tau_proxy", ctypes.c_float),
+                ("tau_jsd", ctypes.c_float), ("k_min_blocks", ctypes.c_int32),
+                ("router", ctypes.c_int32), ("vs_rule", ctypes.c_int32), ("sm_scale", ctypes.c_float)]
+
+    @property
+    def n_blocks(self) -> int:
+        return self.seqlen // self.block
+
+
+def make_params(batch, h_q, h_kv, seqlen, head_dim, block=128, alpha=1.0, gamma=0.95,
+                tau_proxy=0.2, tau_jsd=0.1, k_min_blocks=8, router="cstruct", vs_rule="alpha",
+                sm_scale=0.0) -> CrispParams:
+    return CrispParams(batch, h_q, h_kv, seqlen, head_dim, block, alpha, gamma, tau_proxy, tau_jsd,
+                       k_min_blocks, ROUTER[router] if isinstance(router, str) else int(router),
+                       VS_RULE[vs_rule] if isinstance(vs_rule, str) else int(vs_rule), sm_scale)
+
+
+def params_for(q: torch.Tensor, k: torch.Tensor, **kw) -> CrispParams:
+    b, hq, n, d = q.shape
+    return make_params(b, hq, k.shape[1], n, d, **kw)
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Loads libcrisp.so once and declares the C signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libcrisp.so not built at {path}; run python -m dynamic_block_sparse_qk_b200.build")
+    lib = ctypes.CDLL(path)
+    P = ctypes.POINTER(CrispParams)
+    vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    lib.crisp_version.restype = i32
+    lib.crisp_status_string.restype = ctypes.c_char_p
+    lib.crisp_status_string.argtypes = [i32]
+    lib.crisp_check_params.restype = i32
+    lib.crisp_check_params.argtypes = [P]
+    lib.crisp_workspace_size.restype = sz
+    lib.crisp_workspace_size.argtypes = [P]
+    lib.crisp_route.restype = i32
+    lib.crisp_route.argtypes = [P, vp, vp, vp, sz, vp, vp, vp, vp, vp]
+    lib.crisp_select.restype = i32
+    lib.crisp_select.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp, vp, vp, vp, vp]
+    lib.crisp_sparse_prefill.restype = i32
+    lib.crisp_sparse_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.crisp_dense_prefill.restype = i32
+    lib.crisp_dense_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.crisp_get_device_status.restype = i32
+    lib.crisp_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), vp]
+    _lib = lib
+    return lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(fn: str, status: int):
+    if status != CRISP_OK:
+        raise CrispError(fn, status)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("CRISP tensors must live on a CUDA device")
+        if t is not None and not t.is_contiguous():
+            raise ValueError("CRISP tensors must be contiguous")
+
+
+def crisp_workspace_size(p: CrispParams) -> int:
+    n = load_library().crisp_workspace_size(ctypes.byref(p))
+    if n == 0:
+        _check("crisp_workspace_size", load_library().crisp_check_params(ctypes.byref(p)))
+    return int(n)
+
+
+def alloc_workspace(p: CrispParams, device="cuda") -> torch.Tensor:
+    """Workspace tensor with its status word (first 8 bytes) cleared."""
+    ws = torch.empty(crisp_workspace_size(p), dtype=torch.uint8, device=device)
+    ws[:256].zero_()
+    return ws
+
+
+def crisp_route(p: CrispParams, q, k, ws, pattern=None, score=None, p_v=None, p_s=None, stream=None):
+    """Algorithm 2 for every head. Returns (pattern, score, p_v, p_s)."""
+    _need_cuda(q, k, ws)
+    bh, nb = p.batch * p.h_q, p.n_blocks
+    dev = q.device
+    pattern = torch.empty(bh, dtype=torch.int32, device=dev) if pattern is None else pattern
+    score = torch.empty(bh, dtype=torch.float32, device=dev) if score is None else score
+    p_v = torch.empty(bh, nb, dtype=torch.float32, device=dev) if p_v is None else p_v
+    p_s = torch.empty(bh, nb, dtype=torch.float32, device=dev) if p_s is None else p_s
+    _check("crisp_route", load_library().crisp_route(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(ws), ws.numel(), _ptr(pattern), _ptr(score),
+        _ptr(p_v), _ptr(p_s), _stream(stream)))
+    return pattern, score, p_v, p_s
+
+
+def crisp_select(p: CrispParams, q, k, pattern, p_v, p_s, ws, want_mask=True, mask=None,
+                 tile_idx=None, tile_cnt=None, vs_sel=None, stream=None):
+    """Algorithms 3/4/6 and tile lists. Returns (mask or None, tile_idx, tile_cnt).
+
+    Pass a uint8 tensor [B*H_q, 2, N_b] as ``vs_sel`` to receive the selected
+    vertical / slash block flags of VS heads."""
+    _need_cuda(q, k, pattern, p_v, p_s, ws)
+    bh, nb = p.batch * p.h_q, p.n_blocks
+    dev = q.device
+    if want_mask and mask is None:
+        mask = torch.empty(bh, nb, nb, dtype=torch.uint8, device=dev)
+    tile_idx = torch.empty(bh, nb, nb, dtype=torch.int32, device=dev) if tile_idx is None else tile_idx
+    tile_cnt = torch.empty(bh, nb, dtype=torch.int32, device=dev) if tile_cnt is None else tile_cnt
+    _check("crisp_select", load_library().crisp_select(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(pattern), _ptr(p_v), _ptr(p_s), _ptr(ws), ws.numel(),
+        _ptr(mask), _ptr(vs_sel), _ptr(tile_idx), _ptr(tile_cnt), _stream(stream)))
+    return mask, tile_idx, tile_cnt
+
+
+def crisp_sparse_prefill(p: CrispParams, q, k, v, tile_idx, tile_cnt, ws, o=None, lse=None,
+                         want_lse=True, stream=None):
+    """Eq. 1 over the selected tiles. Returns (o, lse or None)."""
+    _need_cuda(q, k, v, tile_idx, tile_cnt, ws)
+    o = torch.empty_like(q) if o is None else o
+    if want_lse and lse is None:
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    _check("crisp_sparse_prefill", load_library().crisp_sparse_prefill(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(tile_idx), _ptr(tile_cnt), _ptr(o),
+        _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return o, lse
+
+
+def crisp_dense_prefill(p: CrispParams, q, k, v, ws, o=None, lse=None, want_lse=True, stream=None):
+    """Dense causal attention with the same kernel. Returns (o, lse or None)."""
+    _need_cuda(q, k, v, ws)
+    o = torch.empty_like(q) if o is None else o
+    if want_lse and lse is None:
+        lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device)
+    _check("crisp_dense_prefill", load_library().crisp_dense_prefill(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    return o, lse
+
+
+def crisp_get_device_status(ws, stream=None) -> int:
+    st = ctypes.c_int32(0)
+    _check("crisp_get_device_status",
+           load_library().crisp_get_device_status(_ptr(ws), ctypes.byref(st), _stream(stream)))
+    return int(st.value)
+
+
+def crisp_prefill(q, k, v, ws=None, want_mask=False, stream=None, **kw):
+    """Algorithm 1 end to end: route, select, sparse attention.
+
+    Returns a dict with o, lse, pattern, score, p_v, p_s, tile_idx, tile_cnt
+    (and mask when requested)."""
+    p = params_for(q, k, **kw)
+    ws = alloc_workspace(p, q.device) if ws is None else ws
+    pattern, score, p_v, p_s = crisp_route(p, q, k, ws, stream=stream)
+    mask, tile_idx, tile_cnt = crisp_select(p, q, k, pattern, p_v, p_s, ws, want_mask=want_mask,
+                                            stream=stream)
+    o, lse = crisp_sparse_prefill(p, q, k, v, tile_idx, tile_cnt, ws, stream=stream)
+    return {"o": o, "lse": lse, "pattern": pattern, "score": score, "p_v": p_v, "p_s": p_s,
+            "mask": mask, "tile_idx": tile_idx, "tile_cnt": tile_cnt, "params": p, "ws": ws}

@@ -1,0 +1,165 @@
+// Shared device helpers and the workspace layout of the CRISP sm_100a library.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/crisp.h"
+
+namespace crisp {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kMaxBlocks = 8192;  // N_b limit (selection kernels keep one row in smem)
+
+// ----------------------------------------------------------------------------
+// Workspace layout. Every region is 256-byte aligned. The caller allocates
+// `total` bytes once per problem shape; all stages share it in stream order.
+// ----------------------------------------------------------------------------
+struct Workspace {
+  size_t status;      // int32[64]: [0] status word, [1] first bad index, [8..] counters
+  size_t stat_m;      // float[BH][Nb][R]   per-row max of a proxy key tile (log2 units)
+  size_t stat_lo;     // float[BH][Nb][R]   sum exp2(s-m) over tile columns c <= r
+  size_t stat_hi;     // float[BH][Nb][R]   sum exp2(s-m) over tile columns c >  r
+  size_t chunk_m;     // float[BH][NC][R]   per-row max over a chunk of key tiles
+  size_t chunk_l;     // float[BH][NC][R]   per-row sum over the chunk (scaled to chunk_m)
+  size_t row_m;       // float[BH][R]       proxy row max
+  size_t row_l;       // float[BH][R]       proxy row normaliser
+  size_t kbar;        // float[B*Hkv][Nb][d] block means of K
+  size_t qbar;        // float[BH][Nb][d]    block means of Q (PE heads)
+  size_t sel;         // uint8[BH][2][Nb]    selected vertical / slash blocks
+  size_t abar;        // float[BH][Nb][Nb]   PE estimate divided by N_b
+  size_t hist_cnt;    // uint32[BH][4096]    radix-select bucket counts
+  size_t hist_sum;    // double[BH][4096]    radix-select bucket sums
+  size_t pe_state;    // PeState[BH]
+  size_t eq_cnt;      // uint32[BH][Nb]      per-row count of entries equal to the cut value
+  size_t total;
+};
+
+struct PeState {
+  uint32_t prefix;     // decided high bits of the cut value
+  uint32_t all;        // 1 when the whole triangle sums below gamma (select all)
+  uint32_t m_equal;    // how many entries equal to the cut value are taken
+  uint32_t pad;
+  double above_sum;    // sum of entries strictly above the decided range
+};
+
+constexpr int kProxyChunk = 32;  // key tiles per proxy CTA
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+__host__ __device__ inline Workspace make_workspace(const crisp_params& p) {
+  Workspace w{};
+  const size_t BH = size_t(p.batch) * p.h_q;
+  const size_t BK = size_t(p.batch) * p.h_kv;
+  const size_t nb = size_t(p.seqlen / p.block);
+  const size_t R = size_t(p.block);
+  const size_t nc = (nb + kProxyChunk - 1) / kProxyChunk;
+  const size_t d = size_t(p.head_dim);
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
+  w.status = take(64 * 4);
+  w.stat_m = take(BH * nb * R * 4);
+  w.stat_lo = take(BH * nb * R * 4);
+  w.stat_hi = take(BH * nb * R * 4);
+  w.chunk_m = take(BH * nc * R * 4);
+  w.chunk_l = take(BH * nc * R * 4);
+  w.row_m = take(BH * R * 4);
+  w.row_l = take(BH * R * 4);
+  w.kbar = take(BK * nb * d * 4);
+  w.qbar = take(BH * nb * d * 4);
+  w.sel = take(BH * 2 * nb);
+  w.abar = take(BH * nb * nb * 4);
+  w.hist_cnt = take(BH * 4096 * 4);
+  w.hist_sum = take(BH * 4096 * 8);
+  w.pe_state = take(BH * sizeof(PeState));
+  w.eq_cnt = take(BH * nb * 4);
+  w.total = off;
+  return w;
+}
+
+template <typename T>
+__host__ __device__ inline T* ws_ptr(void* base, size_t off) {
+  return reinterpret_cast<T*>(reinterpret_cast<char*>(base) + off);
+}
+
+// Records the first device-side error in the status word (index kept for debugging).
+__device__ inline void report_error(int32_t* status, int32_t code, int32_t where) {
+  if (atomicCAS(status, 0, code) == 0) status[1] = where;
+}
+
+// ----------------------------------------------------------------------------
+// Warp-level helpers.
+// ----------------------------------------------------------------------------
+__device__ inline float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ inline float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ inline double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ inline float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ----------------------------------------------------------------------------
+// Legacy tensor-core (mma.sync m16n8k16 bf16) and async-copy helpers, used by
+// the proxy-score kernel.
+// ----------------------------------------------------------------------------
+__device__ inline uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ inline void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(dst), "l"(src));
+}
+__device__ inline void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+template <int N>
+__device__ inline void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
+
+__device__ inline void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                   uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ inline void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                         uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ inline void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                      uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ inline uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in a tile whose rows are
+// `row_bytes` long, with the chunk index XOR-swizzled by (row % 8).
+__device__ inline uint32_t swz(int row, int chunk, int row_bytes) {
+  return uint32_t(row * row_bytes + ((chunk ^ (row & 7)) << 4));
+}
+
+}  // namespace crisp

@@ -1,0 +1,27 @@
+// Internal launch entry points shared between the translation units of the
+// CRISP library (not part of the public C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/crisp.h"
+
+namespace crisp {
+
+cudaError_t launch_pool(const crisp_params& p, const void* x, int heads, const int32_t* pattern,
+                        int mode, float* out, cudaStream_t st);
+
+cudaError_t run_route(const crisp_params& p, const void* q, const void* k, void* ws,
+                      int32_t* pattern, float* score, float* p_v, float* p_s, cudaStream_t st);
+
+cudaError_t run_select(const crisp_params& p, const void* q, const void* k, const int32_t* pattern,
+                       const float* p_v, const float* p_s, void* ws, uint8_t* mask,
+                       int32_t* tile_idx, int32_t* tile_cnt, cudaStream_t st);
+
+// Block-sparse (tile_idx != NULL) or dense causal attention.
+cudaError_t run_attention(const crisp_params& p, const void* q, const void* k, const void* v,
+                          const int32_t* tile_idx, const int32_t* tile_cnt, void* o, float* lse,
+                          void* ws, cudaStream_t st);
+
+}  // namespace crisp

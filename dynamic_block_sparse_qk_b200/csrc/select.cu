@@ -1,0 +1,524 @@
+// Index selection on sm_100a: the sink-aware VS index (CRISP paper,
+// Algorithm 3, Eq. 3-4), the FlexPrefill gamma VS index (Appendix A,
+// Algorithm 6), the PE index (Algorithm 4) and the tile lists that feed the
+// block-sparse attention kernel.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace crisp {
+
+// ---------------------------------------------------------------------------
+// VS selection, one CTA (1024 threads) per (query head, direction).
+// Scores stay in shared memory. ALPHA: Eq. 4 count, clip, top-k (rank based
+// only when the count is below k_min). GAMMA: rank every block, scatter to
+// descending order, fp64 prefix sum, first prefix >= gamma, clip.
+// Ranks order by value descending, equal values by lower index.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) vs_select_kernel(crisp_params p, const int32_t* pattern,
+                                                         const float* __restrict__ p_v,
+                                                         const float* __restrict__ p_s, void* ws) {
+  extern __shared__ unsigned char sm[];
+  const int nb = p.seqlen / p.block;
+  float* pv = reinterpret_cast<float*>(sm);                 // [nb]
+  float* sorted = pv + nb;                                   // [nb] (GAMMA)
+  double* scan = reinterpret_cast<double*>(sorted + nb);  // [1024], 8-byte aligned (2*nb floats)
+  __shared__ int cnt_s, kcut_s;
+  const Workspace W = make_workspace(p);
+  const int bh = blockIdx.x, dir = blockIdx.y;
+  const float* src = (dir == 0 ? p_v : p_s) + size_t(bh) * nb;
+  uint8_t* sel = ws_ptr<uint8_t>(ws, W.sel) + (size_t(bh) * 2 + dir) * nb;
+  const int tid = threadIdx.x;
+  if (pattern[bh] != CRISP_PATTERN_VS) {
+    for (int j = tid; j < nb; j += 1024) sel[j] = 0;
+    return;
+  }
+  for (int j = tid; j < nb; j += 1024) pv[j] = src[j];
+  if (tid == 0) { cnt_s = 0; kcut_s = nb; }
+  __syncthreads();
+  auto rank_of = [&](int j) {
+    const float x = pv[j];
+    int rk = 0;
+    for (int i = 0; i < nb; ++i) {
+      const float y = pv[i];
+      rk += (y > x) || (y == x && i < j);
+    }
+    return rk;
+  };
+  int k;
+  if (p.vs_rule == CRISP_VS_ALPHA) {
+    float r = (1.0f - pv[0]) - pv[nb - 1];
+    r = fmaxf(r, 0.0f);
+    const float mu = r / float(nb - 2);
+    const float thr = p.alpha * mu;
+    int c = 0;
+    for (int j = tid; j < nb; j += 1024) c += pv[j] > thr;
+    c = __reduce_add_sync(0xffffffffu, c);
+    if ((tid & 31) == 0) atomicAdd(&cnt_s, c);
+    __syncthreads();
+    const int cnt = cnt_s;
+    k = min(max(cnt, p.k_min_blocks), nb);
+    if (k == cnt) {
+      for (int j = tid; j < nb; j += 1024) sel[j] = pv[j] > thr;
+      return;
+    }
+    for (int j = tid; j < nb; j += 1024) sel[j] = rank_of(j) < k;
+    return;
+  }
+  // GAMMA (Algorithm 6).
+  for (int j = tid; j < nb; j += 1024) sorted[rank_of(j)] = pv[j];
+  __syncthreads();
+  // Block-wide inclusive prefix sum in fp64: thread t owns a contiguous run.
+  const int per = (nb + 1023) / 1024;
+  const int j0 = tid * per, j1 = min(j0 + per, nb);
+  double run = 0.0;
+  for (int j = j0; j < j1; ++j) run += double(sorted[j]);
+  scan[tid] = run;
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {
+    const double v = tid >= off ? scan[tid - off] : 0.0;
+    __syncthreads();
+    scan[tid] += v;
+    __syncthreads();
+  }
+  double acc = tid > 0 ? scan[tid - 1] : 0.0;
+  const double g = double(p.gamma);
+  for (int j = j0; j < j1; ++j) {
+    acc += double(sorted[j]);
+    if (acc >= g) { atomicMin(&kcut_s, j + 1); break; }
+  }
+  __syncthreads();
+  k = min(max(kcut_s, p.k_min_blocks), nb);
+  for (int j = tid; j < nb; j += 1024) sel[j] = rank_of(j) < k;
+}
+
+// ---------------------------------------------------------------------------
+// PE estimate (Algorithm 4 line 4): logits of Q_bar K_bar^T for kb <= qb,
+// 64x64 tiles per CTA, fp32 FMA; written in log2 units into abar together
+// with per-(row, tile) max / sum partials. Then a row pass normalises and
+// divides by N_b (Algorithm 4 line 6: the total of N_b causal rows is N_b).
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) pe_logits_kernel(crisp_params p, const int32_t* pattern,
+                                                        void* ws) {
+  constexpr int T = 64, KC = 32;
+  __shared__ float qs[KC][T + 1];
+  __shared__ float kst[KC][T + 1];
+  __shared__ float rmax[T][17], rsum[T][17];
+  const Workspace W = make_workspace(p);
+  const int nb = p.seqlen / p.block;
+  const int bh = blockIdx.z;
+  if (pattern[bh] != CRISP_PATTERN_PE) return;
+  const int tq = blockIdx.y, tk = blockIdx.x;
+  if (tk > tq) return;
+  const int b = bh / p.h_q, h = bh % p.h_q, hk = h / (p.h_q / p.h_kv);
+  const float* qbar = ws_ptr<float>(ws, W.qbar) + size_t(bh) * nb * D;
+  const float* kbar = ws_ptr<float>(ws, W.kbar) + (size_t(b) * p.h_kv + hk) * nb * D;
+  float* abar = ws_ptr<float>(ws, W.abar) + size_t(bh) * nb * nb;
+  const float sl2 = (p.sm_scale > 0.f ? p.sm_scale : rsqrtf(float(D))) * kLog2e;
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;   // 4x4 micro-tile per thread
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < D; k0 += KC) {
+    for (int i = tid; i < T * KC; i += 256) {
+      const int r = i / KC, c = i % KC;
+      const int qr = tq * T + r, kr = tk * T + r;
+      qs[c][r] = qr < nb ? qbar[size_t(qr) * D + k0 + c] : 0.f;
+      kst[c][r] = kr < nb ? kbar[size_t(kr) * D + k0 + c] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int c = 0; c < KC; ++c) {
+      float a[4], bb[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) { a[i] = qs[c][ty * 4 + i]; bb[i] = kst[c][tx * 4 + i]; }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+  // write logits (log2 units) and per-row partial max / sum over this tile
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int qb = tq * T + ty * 4 + i;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int kb = tk * T + tx * 4 + j;
+      const bool ok = qb < nb && kb <= qb;
+      acc[i][j] = ok ? acc[i][j] * sl2 : -INFINITY;
+      if (ok) abar[size_t(qb) * nb + kb] = acc[i][j];
+      mx = fmaxf(mx, acc[i][j]);
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) s += (acc[i][j] == -INFINITY) ? 0.f : exp2f(acc[i][j] - mx);
+    rmax[ty * 4 + i][tx] = mx;
+    rsum[ty * 4 + i][tx] = s;
+  }
+  __syncthreads();
+  if (tid < T) {
+    const int qb = tq * T + tid;
+    if (qb < nb) {
+      float mx = -INFINITY;
+      for (int j = 0; j < 16; ++j) mx = fmaxf(mx, rmax[tid][j]);
+      float s = 0.f;
+      for (int j = 0; j < 16; ++j)
+        if (rmax[tid][j] != -INFINITY) s += rsum[tid][j] * exp2f(rmax[tid][j] - mx);
+      const int ntile = (nb + T - 1) / T;
+      // partials reuse the proxy statistic regions (free once routing is done)
+      ws_ptr<float>(ws, W.stat_m)[(size_t(bh) * nb + qb) * ntile + tk] = mx;
+      ws_ptr<float>(ws, W.stat_lo)[(size_t(bh) * nb + qb) * ntile + tk] = s;
+    }
+  }
+}
+
+// One warp per PE row: combine partials, rewrite abar[qb][kb] = softmax / N_b.
+__global__ void pe_normalize_kernel(crisp_params p, const int32_t* pattern, void* ws) {
+  const Workspace W = make_workspace(p);
+  const int nb = p.seqlen / p.block;
+  const int bh = blockIdx.y;
+  if (pattern[bh] != CRISP_PATTERN_PE) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qb = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (qb >= nb) return;
+  const int ntile = (nb + 63) / 64;
+  const int nt = qb / 64 + 1;
+  const float* pm = ws_ptr<float>(ws, W.stat_m) + (size_t(bh) * nb + qb) * ntile;
+  const float* ps = ws_ptr<float>(ws, W.stat_lo) + (size_t(bh) * nb + qb) * ntile;
+  float mx = -INFINITY;
+  for (int t = lane; t < nt; t += 32) mx = fmaxf(mx, pm[t]);
+  mx = warp_max(mx);
+  float s = 0.f;
+  for (int t = lane; t < nt; t += 32) s += ps[t] * exp2f(pm[t] - mx);
+  s = warp_sum(s);
+  const float inv = 1.0f / (s * float(nb));
+  float* row = ws_ptr<float>(ws, W.abar) + (size_t(bh) * nb + qb) * nb;
+  for (int kb = lane; kb <= qb; kb += 32) row[kb] = exp2f(row[kb] - mx) * inv;
+}
+
+// ---------------------------------------------------------------------------
+// Gamma cut over the PE triangle by radix select on the float bit patterns
+// (positive floats order like their bits). Level 0: bits 31..20, level 1:
+// bits 19..8, level 2: bits 7..0. Bucket counts and fp64 sums per head.
+// ---------------------------------------------------------------------------
+__device__ inline void level_geom(int level, int& shift, int& nbk) {
+  shift = level == 0 ? 20 : (level == 1 ? 8 : 0);
+  nbk = level == 2 ? 256 : 4096;
+}
+
+__global__ void __launch_bounds__(256) pe_hist_kernel(crisp_params p, const int32_t* pattern,
+                                                      void* ws, int level) {
+  __shared__ uint32_t hc[4096];
+  __shared__ double hs[4096];
+  const Workspace W = make_workspace(p);
+  const int nb = p.seqlen / p.block;
+  const int bh = blockIdx.y;
+  if (pattern[bh] != CRISP_PATTERN_PE) return;
+  const PeState st = ws_ptr<PeState>(ws, W.pe_state)[bh];
+  if (st.all) return;
+  int shift, nbk;
+  level_geom(level, shift, nbk);
+  for (int i = threadIdx.x; i < nbk; i += 256) { hc[i] = 0; hs[i] = 0.0; }
+  __syncthreads();
+  const float* abar = ws_ptr<float>(ws, W.abar) + size_t(bh) * nb * nb;
+  const int rows_per = 8;
+  const int q0 = blockIdx.x * rows_per, q1 = min(q0 + rows_per, nb);
+  const uint32_t hi_shift = shift + (level == 2 ? 8 : 12);
+  for (int qb = q0; qb < q1; ++qb) {
+    const float* row = abar + size_t(qb) * nb;
+    for (int kb = threadIdx.x; kb <= qb; kb += 256) {
+      const float v = row[kb];
+      const uint32_t u = __float_as_uint(v);
+      if (level > 0 && (u >> hi_shift) != (st.prefix >> hi_shift)) continue;
+      const uint32_t bk = (u >> shift) & uint32_t(nbk - 1);
+      atomicAdd(&hc[bk], 1u);
+      atomicAdd(&hs[bk], double(v));
+    }
+  }
+  __syncthreads();
+  uint32_t* gc = ws_ptr<uint32_t>(ws, W.hist_cnt) + size_t(bh) * 4096;
+  double* gs = ws_ptr<double>(ws, W.hist_sum) + size_t(bh) * 4096;
+  for (int i = threadIdx.x; i < nbk; i += 256)
+    if (hc[i]) { atomicAdd(&gc[i], hc[i]); atomicAdd(&gs[i], hs[i]); }
+}
+
+// One CTA (1024 threads) per PE head: the highest bucket whose descending
+// cumulative sum (above_sum + buckets above + itself) reaches gamma.
+__global__ void __launch_bounds__(1024) pe_find_kernel(crisp_params p, const int32_t* pattern,
+                                                       void* ws, int level) {
+  __shared__ double suf[1024];
+  __shared__ int best, lowest;
+  const Workspace W = make_workspace(p);
+  const int bh = blockIdx.x;
+  if (pattern[bh] != CRISP_PATTERN_PE) return;
+  PeState* stp = ws_ptr<PeState>(ws, W.pe_state) + bh;
+  if (stp->all) return;
+  int shift, nbk;
+  level_geom(level, shift, nbk);
+  uint32_t* gc = ws_ptr<uint32_t>(ws, W.hist_cnt) + size_t(bh) * 4096;
+  double* gs = ws_ptr<double>(ws, W.hist_sum) + size_t(bh) * 4096;
+  const int tid = threadIdx.x;
+  const int per = nbk / 1024 > 0 ? nbk / 1024 : 1;   // 4 (levels 0,1) or 1 (level 2)
+  // thread t owns buckets [hi .. lo] counted from the top: top index = nbk-1 - t*per
+  double own = 0.0;
+  for (int i = 0; i < per; ++i) {
+    const int bk = nbk - 1 - (tid * per + i);
+    if (bk >= 0) own += gs[bk];
+  }
+  suf[tid] = own;
+  if (tid == 0) { best = -1; lowest = 1 << 30; }
+  __syncthreads();
+  for (int bk = tid; bk < nbk; bk += 1024)
+    if (gc[bk]) atomicMin(&lowest, bk);
+  for (int off = 1; off < 1024; off <<= 1) {
+    const double v = tid >= off ? suf[tid - off] : 0.0;
+    __syncthreads();
+    suf[tid] += v;
+    __syncthreads();
+  }
+  const double g = double(p.gamma);
+  const double above0 = stp->above_sum;
+  double run = above0 + (tid > 0 ? suf[tid - 1] : 0.0);
+  for (int i = 0; i < per; ++i) {
+    const int bk = nbk - 1 - (tid * per + i);
+    if (bk < 0) break;
+    if (run + gs[bk] >= g) { atomicMax(&best, bk); break; }
+    run += gs[bk];
+  }
+  __syncthreads();
+  // Recompute the sum strictly above the chosen bucket (single thread, exact order).
+  if (tid == 0) {
+    PeState s = *stp;
+    int cut = best;
+    if (cut < 0 && level > 0 && lowest < nbk) cut = lowest;  // rounding fell short: whole range
+    if (cut < 0) {
+      s.all = 1;                       // the whole triangle sums below gamma
+    } else {
+      const int best = cut;
+      double above = above0;
+      for (int bk = nbk - 1; bk > best; --bk) above += gs[bk];
+      s.prefix |= uint32_t(best) << shift;
+      s.above_sum = above;
+      if (level == 2) {
+        const float tv = __uint_as_float(s.prefix);
+        const double need = g - above;
+        double m = ceil(need / double(tv));
+        if (m < 1.0) m = 1.0;
+        const double cap = double(gc[best]);
+        if (m > cap) m = cap;
+        s.m_equal = uint32_t(m);
+      }
+    }
+    *stp = s;
+  }
+  __syncthreads();
+  for (int i = tid; i < nbk; i += 1024) { gc[i] = 0; gs[i] = 0.0; }
+}
+
+// Per-row count of entries equal to the cut value, then an exclusive scan
+// per head, so the tile builder can take the first m_equal of them in flat
+// (row-major) order.
+__global__ void pe_eqcount_kernel(crisp_params p, const int32_t* pattern, void* ws) {
+  const Workspace W = make_workspace(p);
+  const int nb = p.seqlen / p.block;
+  const int bh = blockIdx.y;
+  if (pattern[bh] != CRISP_PATTERN_PE) return;
+  const PeState st = ws_ptr<PeState>(ws, W.pe_state)[bh];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qb = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (qb >= nb || st.all) return;
+  const float tv = __uint_as_float(st.prefix);
+  const float* row = ws_ptr<float>(ws, W.abar) + (size_t(bh) * nb + qb) * nb;
+  uint32_t c = 0;
+  for (int kb = lane; kb <= qb; kb += 32) c += row[kb] == tv;
+  c = __reduce_add_sync(0xffffffffu, c);
+  if (lane == 0) ws_ptr<uint32_t>(ws, W.eq_cnt)[size_t(bh) * nb + qb] = c;
+}
+
+__global__ void __launch_bounds__(1024) pe_eqscan_kernel(crisp_params p, const int32_t* pattern,
+                                                         void* ws) {
+  __shared__ uint32_t part[1024];
+  const Workspace W = make_workspace(p);
+  const int nb = p.seqlen / p.block;
+  const int bh = blockIdx.x;
+  if (pattern[bh] != CRISP_PATTERN_PE) return;
+  if (ws_ptr<PeState>(ws, W.pe_state)[bh].all) return;
+  uint32_t* ec = ws_ptr<uint32_t>(ws, W.eq_cnt) + size_t(bh) * nb;
+  const int tid = threadIdx.x;
+  const int per = (nb + 1023) / 1024;
+  const int j0 = tid * per, j1 = min(j0 + per, nb);
+  uint32_t s = 0;
+  for (int j = j0; j < j1; ++j) s += ec[j];
+  part[tid] = s;
+  __syncthreads();
+  for (int off = 1; off < 1024; off <<= 1) {
+    const uint32_t v = tid >= off ? part[tid - off] : 0u;
+    __syncthreads();
+    part[tid] += v;
+    __syncthreads();
+  }
+  uint32_t run = tid > 0 ? part[tid - 1] : 0u;
+  for (int j = j0; j < j1; ++j) {
+    const uint32_t c = ec[j];
+    ec[j] = run;
+    run += c;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Tile lists: one warp per (head, query block). Lanes cover 4 consecutive
+// key blocks per step (uchar4 mask stores), a warp scan compacts the active
+// ids in ascending order.
+// VS: tile active iff kb in S_v u {0}, or qb-kb or qb-kb-1 in the offset set
+//     O = {N_b-1-j : j in S_s} u {0}.
+// PE: active iff chosen by the gamma cut, or kb == qb, or kb == 0.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) build_tiles_kernel(crisp_params p, const int32_t* pattern,
+                                                          void* ws, uint8_t* __restrict__ mask,
+                                                          int32_t* __restrict__ tile_idx,
+                                                          int32_t* __restrict__ tile_cnt) {
+  const Workspace W = make_workspace(p);
+  const int nb = p.seqlen / p.block;
+  const int bh = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qb = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (qb >= nb) return;
+  const bool vs = pattern[bh] == CRISP_PATTERN_VS;
+  const uint8_t* sv = ws_ptr<uint8_t>(ws, W.sel) + size_t(bh) * 2 * nb;
+  const uint8_t* ss = sv + nb;
+  PeState st{};
+  const float* arow = nullptr;
+  uint32_t eq_before = 0;
+  float tv = 0.f;
+  if (!vs) {
+    st = ws_ptr<PeState>(ws, W.pe_state)[bh];
+    arow = ws_ptr<float>(ws, W.abar) + (size_t(bh) * nb + qb) * nb;
+    tv = __uint_as_float(st.prefix);
+    if (!st.all) eq_before = ws_ptr<uint32_t>(ws, W.eq_cnt)[size_t(bh) * nb + qb];
+  }
+  auto offset_on = [&](int o) -> bool {
+    if (o == 0) return true;
+    if (o < 0 || o >= nb) return false;
+    return ss[nb - 1 - o] != 0;
+  };
+  int32_t* idx = tile_idx + (size_t(bh) * nb + qb) * nb;
+  uint8_t* mrow = mask ? mask + (size_t(bh) * nb + qb) * nb : nullptr;
+  int count = 0;
+  uint32_t eq_seen = eq_before;
+  for (int base = 0; base < nb; base += 128) {
+    bool f[4];
+    int neq = 0;
+    bool isq[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int kb = base + lane * 4 + i;
+      bool on = false;
+      isq[i] = false;
+      if (kb <= qb) {
+        if (vs) {
+          const int dlt = qb - kb;
+          on = kb == 0 || sv[kb] || offset_on(dlt) || offset_on(dlt - 1);
+        } else {
+          on = kb == 0 || kb == qb || st.all;
+          if (!st.all) {
+            const float v = arow[kb];
+            if (v > tv) on = true;
+            else if (v == tv) { isq[i] = true; ++neq; }
+          }
+        }
+      }
+      f[i] = on;
+    }
+    if (!vs && !st.all) {
+      // rank of this lane's equal entries among all equal entries in flat order
+      uint32_t pre = neq;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xffffffffu, pre, o);
+        if (lane >= o) pre += v;
+      }
+      uint32_t rank = eq_seen + pre - neq;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (isq[i]) { if (rank < st.m_equal) f[i] = true; ++rank; }
+      eq_seen += __shfl_sync(0xffffffffu, pre, 31);
+    }
+    if (mrow) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (base + lane * 4 + i < nb) mrow[base + lane * 4 + i] = f[i];
+    }
+    int c = int(f[0]) + int(f[1]) + int(f[2]) + int(f[3]);
+    int pre = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, pre, o);
+      if (lane >= o) pre += v;
+    }
+    int pos = count + pre - c;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if (f[i]) idx[pos++] = base + lane * 4 + i;
+    count += __shfl_sync(0xffffffffu, pre, 31);
+    if (base + 128 > qb) {
+      // the rest of the row lies above the diagonal: mask zeros only
+      for (int b2 = base + 128 + lane; mrow && b2 < nb; b2 += 32) mrow[b2] = 0;
+      break;
+    }
+  }
+  if (lane == 0) tile_cnt[size_t(bh) * nb + qb] = count;
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+cudaError_t run_select(const crisp_params& p, const void* q, const void* k, const int32_t* pattern,
+                       const float* p_v, const float* p_s, void* ws, uint8_t* mask,
+                       int32_t* tile_idx, int32_t* tile_cnt, cudaStream_t st) {
+  const Workspace W = make_workspace(p);
+  const int nb = p.seqlen / p.block;
+  const int BH = p.batch * p.h_q;
+  cudaError_t e;
+  // (1) VS selection per direction.
+  {
+    const size_t smem = size_t(nb) * 8 + 1024 * 8;
+    cudaFuncSetAttribute(vs_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    vs_select_kernel<<<dim3(BH, 2), 1024, smem, st>>>(p, pattern, p_v, p_s, ws);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // (2) PE path: pooling, estimate, gamma cut.
+  if (p.router != CRISP_ROUTER_JSD) {
+    e = launch_pool(p, k, p.batch * p.h_kv, pattern, 0, ws_ptr<float>(ws, W.kbar), st);
+    if (e != cudaSuccess) return e;
+  }
+  e = launch_pool(p, q, BH, pattern, 1, ws_ptr<float>(ws, W.qbar), st);
+  if (e != cudaSuccess) return e;
+  {
+    const int nt = (nb + 63) / 64;
+    dim3 grid(nt, nt, BH);
+    if (p.head_dim == 64) pe_logits_kernel<64><<<grid, 256, 0, st>>>(p, pattern, ws);
+    else pe_logits_kernel<128><<<grid, 256, 0, st>>>(p, pattern, ws);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    pe_normalize_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, pattern, ws);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if ((e = cudaMemsetAsync(ws_ptr<char>(ws, W.hist_cnt), 0, size_t(BH) * 4096 * 4, st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(ws_ptr<char>(ws, W.hist_sum), 0, size_t(BH) * 4096 * 8, st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(ws_ptr<char>(ws, W.pe_state), 0, size_t(BH) * sizeof(PeState), st)) != cudaSuccess) return e;
+  for (int level = 0; level < 3; ++level) {
+    pe_hist_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, pattern, ws, level);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    pe_find_kernel<<<BH, 1024, 0, st>>>(p, pattern, ws, level);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  pe_eqcount_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, pattern, ws);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  pe_eqscan_kernel<<<BH, 1024, 0, st>>>(p, pattern, ws);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // (3) tile lists.
+  build_tiles_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, pattern, ws, mask, tile_idx, tile_cnt);
+  return cudaGetLastError();
+}
+
+}  // namespace crisp

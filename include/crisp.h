@@ -1,0 +1,143 @@
+/*
+ * crisp.h — C ABI of the B200 (sm_100a) CRISP sparse-prefill library.
+ *
+ * The operation is CRISP sparse attention prefill as defined by the paper
+ * "CRISP: Cliff-awaRe Input-adaptive Sparse Prefilling with
+ * Structural-Mass-Motivated Routing": Algorithm 1 (route each head, select a
+ * sparse index set, attend over it), with PatSearch (Algorithm 2), the
+ * sink-aware VS index (Algorithm 3, Eq. 3-4), the PE index (Algorithm 4),
+ * the FlexPrefill JSD router and gamma VS index kept as comparison paths
+ * (Appendix A, Algorithms 5-6) and block-sparse attention (Eq. 1).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors q, k, v, o are DEVICE pointers to contiguous bf16 arrays of
+ *    layout [batch][heads][seqlen][head_dim] (heads = h_q for q and o,
+ *    h_kv for k and v). GQA: query head h reads KV head h / (h_q / h_kv).
+ *    Every pointer must be 16-byte aligned.
+ *  - The caller owns all memory, including the workspace `ws` of
+ *    `ws_bytes` >= crisp_workspace_size(p) bytes (256-byte aligned). The
+ *    library allocates no device memory and keeps no global state.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream). The return value covers argument validation and
+ *    launch errors only; kernel-side errors (a bounded wait that ran out,
+ *    an out-of-range tile index) are recorded in a status word held in the
+ *    first 8 bytes of `ws`, read back (and cleared) with
+ *    crisp_get_device_status(). crisp_route and crisp_dense_prefill start a
+ *    prefill and clear the word; a caller who runs crisp_select or
+ *    crisp_sparse_prefill alone on a new workspace zeroes those 8 bytes.
+ *  - Block geometry: N_b = seqlen / block. seqlen must be a multiple of 128
+ *    and of block; block is 64 or 128; head_dim is 64 or 128; N_b >= 3.
+ *  - Return codes: CRISP_OK, or a negative crisp_status. Invalid arguments
+ *    never launch a kernel.
+ */
+#ifndef CRISP_H_
+#define CRISP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CRISP_OK = 0,
+  CRISP_ERR_ARG = -1,        /* null pointer, misaligned pointer, bad enum or hyper-parameter */
+  CRISP_ERR_SHAPE = -2,      /* unsupported or inconsistent shape */
+  CRISP_ERR_WORKSPACE = -3,  /* workspace smaller than crisp_workspace_size() */
+  CRISP_ERR_CUDA = -4,       /* a CUDA runtime call or kernel launch failed */
+  CRISP_ERR_TIMEOUT = -5,    /* device status: a bounded wait inside a kernel ran out */
+  CRISP_ERR_DEVICE = -6      /* device status: a kernel found an out-of-range index */
+} crisp_status;
+
+typedef enum { CRISP_ROUTER_CSTRUCT = 0, CRISP_ROUTER_JSD = 1 } crisp_router;
+typedef enum { CRISP_VS_ALPHA = 0, CRISP_VS_GAMMA = 1 } crisp_vs_rule;
+typedef enum { CRISP_PATTERN_VS = 0, CRISP_PATTERN_PE = 1 } crisp_pattern;
+
+/* Problem and hyper-parameters (CRISP paper, Section 5 Setup: tau_proxy 0.2,
+ * gamma 0.95 for PE, alpha 1.0, block 128, k_min 8 blocks per direction). */
+typedef struct {
+  int32_t batch, h_q, h_kv, seqlen, head_dim, block;
+  float alpha;         /* noise-floor multiplier of Eq. 4 (> 0) */
+  float gamma;         /* cumulative coverage of Algorithms 4 and 6, in (0, 1] */
+  float tau_proxy;     /* C_struct routing threshold of Algorithm 2 */
+  float tau_jsd;       /* JSD routing threshold of Algorithm 5 (not given by the paper) */
+  int32_t k_min_blocks;/* minimum blocks per VS direction (Algorithm 3 line 11), >= 1 */
+  int32_t router;      /* crisp_router */
+  int32_t vs_rule;     /* crisp_vs_rule */
+  float sm_scale;      /* softmax scale; 0 selects 1/sqrt(head_dim) */
+} crisp_params;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int crisp_version(void);
+
+/* Human-readable name of a crisp_status value (static string). */
+const char* crisp_status_string(int status);
+
+/* Validates `p` without launching anything. Returns CRISP_OK or the error. */
+int crisp_check_params(const crisp_params* p);
+
+/* Workspace bytes needed by route, select and the prefill kernels for `p`
+ * (0 when `p` is invalid). One workspace may serve all calls of a prefill
+ * issued in order on one stream. */
+size_t crisp_workspace_size(const crisp_params* p);
+
+/* Stage (a)+(b) of Algorithm 1: PatSearch (Algorithm 2) for every head.
+ * Computes the causal proxy map of the last `block` query rows against all
+ * keys without materialising it, its block scores
+ *   p_v[b][h][N_b]  (vertical: per-key mean over proxy rows, block sums),
+ *   p_s[b][h][N_b]  (slash: per-diagonal means, block sums; diagonal of
+ *                    entry (r, j) indexed by j + block - 1 - r),
+ * and routes each head: pattern[b*h_q+h] = CRISP_PATTERN_VS iff
+ *   C_struct = p_v[0] + p_v[N_b-1] >= tau_proxy      (router CSTRUCT, Eq. 2)
+ *   D_JS(p_v, pooled estimate) >= tau_jsd              (router JSD, Algorithm 5).
+ * score[b*h_q+h] receives C_struct or D_JS. All outputs are device arrays
+ * (pattern int32, the rest float32); none may be NULL. */
+int crisp_route(const crisp_params* p, const void* q, const void* k, void* ws, size_t ws_bytes,
+                int32_t* pattern, float* score, float* p_v, float* p_s, void* stream);
+
+/* Stage (c): index selection and tile lists.
+ * VS heads: per direction, Algorithm 3 (vs_rule ALPHA: blocks with
+ * p > alpha*mu, mu = max(1-p[0]-p[N_b-1],0)/(N_b-2), count clipped to
+ * [k_min, N_b], top-k by score, ties to the lower block) or Algorithm 6
+ * (vs_rule GAMMA: smallest prefix of the descending scores reaching gamma,
+ * clipped the same way); the union with vertical block 0 and slash block
+ * N_b-1 marks tile (qb, kb <= qb) iff kb is a selected vertical block or
+ * qb-kb or qb-kb-1 is a selected slash offset (offset = N_b-1-slash id).
+ * PE heads: Algorithm 4 — block-mean pooling of Q and K, causal block
+ * softmax, entries divided by N_b, smallest descending prefix reaching
+ * gamma (ties to the lower flat id qb*N_b+kb), plus tiles (qb,qb), (qb,0).
+ * Outputs (device): tile_cnt[b][h][N_b] (int32) and tile_idx[b][h][N_b][N_b]
+ * (int32; row (b,h,qb) holds tile_cnt ascending key-block ids, the rest
+ * undefined); mask[b][h][N_b][N_b] (uint8 0/1, upper triangle 0) unless
+ * mask == NULL; vs_sel[b][h][2][N_b] (uint8 0/1: selected vertical, then
+ * slash blocks; all 0 for PE heads) unless vs_sel == NULL.
+ * pattern, p_v, p_s are crisp_route's outputs. */
+int crisp_select(const crisp_params* p, const void* q, const void* k, const int32_t* pattern,
+                 const float* p_v, const float* p_s, void* ws, size_t ws_bytes, uint8_t* mask,
+                 uint8_t* vs_sel, int32_t* tile_idx, int32_t* tile_cnt, void* stream);
+
+/* Stage (d): causal GQA block-sparse attention, Eq. 1, over the tiles
+ * listed by crisp_select (whole tiles; token-level causal mask inside).
+ * o: bf16 [b][h_q][seqlen][head_dim]. lse (may be NULL): float32
+ * [b][h_q][seqlen], natural-log sum of exp of the scaled logits. */
+int crisp_sparse_prefill(const crisp_params* p, const void* q, const void* k, const void* v,
+                         const int32_t* tile_idx, const int32_t* tile_cnt, void* o, float* lse,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* Dense causal attention with the same kernel over every causal tile (the
+ * paper's exact-attention baseline, Section 5). Same layouts as above. */
+int crisp_dense_prefill(const crisp_params* p, const void* q, const void* k, const void* v,
+                        void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, copies the device status word out of `ws` into
+ * *status (CRISP_OK or CRISP_ERR_TIMEOUT / CRISP_ERR_DEVICE) and clears it.
+ * Returns CRISP_OK unless the copy itself failed. */
+int crisp_get_device_status(void* ws, int32_t* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CRISP_H_ */

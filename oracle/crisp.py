@@ -262,15 +262,19 @@ def vs_tile_mask(s_v: Sequence[int], s_s: Sequence[int], nb: int) -> np.ndarray:
     ob = N_b - 1 - jb, which meet tile (qb, kb) exactly when qb - kb is ob or
     ob + 1. Tiles are computed whole (plus the causal mask in-tile).
     """
-    mask = np.zeros((nb, nb), dtype=bool)
-    cols = set(int(x) for x in s_v) | {0}
-    offs = set(nb - 1 - int(x) for x in s_s) | {0}
-    for qb in range(nb):
-        for kb in range(qb + 1):
-            dlt = qb - kb
-            if kb in cols or dlt in offs or (dlt - 1) in offs:
-                mask[qb, kb] = True
-    return mask
+    col = np.zeros(nb, dtype=bool)
+    col[np.asarray(s_v, dtype=np.int64)] = True
+    col[0] = True
+    off = np.zeros(nb + 1, dtype=bool)          # off[o]: offset block o selected
+    off[nb - 1 - np.asarray(s_s, dtype=np.int64)] = True
+    off[0] = True
+    qb = np.arange(nb)[:, None]
+    kb = np.arange(nb)[None, :]
+    dlt = qb - kb
+    causal = dlt >= 0
+    d0 = np.where(causal, dlt, nb)              # index nb is always False
+    d1 = np.where(dlt >= 1, dlt - 1, nb)
+    return causal & (col[None, :] | off[d0] | off[d1])
 
 
 def vs_tile_mask_tokenwise(s_v, s_s, n: int, block: int) -> np.ndarray:

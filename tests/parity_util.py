@@ -1,0 +1,192 @@
+"""GPU-vs-oracle comparison with the exemption protocol.
+
+Decisions are compared exactly except for items whose oracle score lies
+within EXEMPT_REL (1e-4) relative of the threshold that decides them
+(counted and returned); attention is compared against the oracle run on the
+GPU's own tile mask: max-abs <= 2e-2 and mean-abs <= 2e-3.
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Optional, Sequence
+
+import numpy as np
+import torch
+
+import oracle as O
+
+EXEMPT_REL = 1e-4
+ATTN_MAX_ABS = 2e-2
+ATTN_MEAN_ABS = 2e-3
+
+
+def run_gpu(w, q, k, v, router="cstruct", vs_rule="alpha", alpha=1.0, gamma=0.95, tau_jsd=0.1):
+    """Runs route -> select -> sparse prefill through the C ABI; returns CPU copies."""
+    import dynamic_block_sparse_qk_b200 as C
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    p = C.params_for(qd, kd, block=w.block, alpha=alpha, gamma=gamma, router=router,
+                     vs_rule=vs_rule, tau_jsd=tau_jsd)
+    ws = C.alloc_workspace(p, qd.device)
+    pattern, score, p_v, p_s = C.crisp_route(p, qd, kd, ws)
+    nb = p.n_blocks
+    vs_sel = torch.empty(p.batch * p.h_q, 2, nb, dtype=torch.uint8, device=qd.device)
+    mask, tidx, tcnt = C.crisp_select(p, qd, kd, pattern, p_v, p_s, ws, want_mask=True, vs_sel=vs_sel)
+    o, lse = C.crisp_sparse_prefill(p, qd, kd, vd, tidx, tcnt, ws)
+    status = C.crisp_get_device_status(ws)
+    out = {"pattern": pattern, "score": score, "p_v": p_v, "p_s": p_s, "vs_sel": vs_sel,
+           "mask": mask, "tile_idx": tidx, "tile_cnt": tcnt, "o": o, "lse": lse}
+    out = {key: val.cpu() for key, val in out.items()}
+    out["status"] = status
+    out["params"] = p
+    del qd, kd, vd, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def oracle_params(w, router="cstruct", vs_rule="alpha", alpha=1.0, gamma=0.95, tau_jsd=0.1):
+    return O.CrispParams(block=w.block, alpha=alpha, gamma=gamma, router=router, vs_rule=vs_rule,
+                         tau_jsd=tau_jsd)
+
+
+def _near(x, ref):
+    return abs(float(x) - float(ref)) <= EXEMPT_REL * abs(float(ref))
+
+
+def vs_exempt(p: np.ndarray, rule: str, alpha: float, gamma: float, k_min: int) -> np.ndarray:
+    """Blocks whose selection could flip under float rounding (one direction)."""
+    p32 = p.astype(np.float32)
+    nb = p32.shape[0]
+    order = np.lexsort((np.arange(nb), -p32.astype(np.float64)))
+    ex = np.zeros(nb, dtype=bool)
+    if rule == "alpha":
+        thr = np.float32(np.float32(alpha) * O.noise_floor(p))
+        ex |= np.abs(p32 - thr) <= EXEMPT_REL * abs(thr)
+        cnt = int(np.count_nonzero(p32 > thr))
+        if cnt < k_min + int(ex.sum()) and k_min <= nb:
+            vk = p32[order[min(k_min, nb) - 1]]
+            ex |= np.abs(p32 - vk) <= EXEMPT_REL * abs(vk)
+    else:
+        cs = np.cumsum(p32[order].astype(np.float64))
+        g = np.float64(np.float32(gamma))
+        hit = np.nonzero(cs >= g)[0]
+        kstar = int(hit[0]) + 1 if hit.size else nb
+        k = min(max(kstar, k_min), nb)
+        vk = p32[order[k - 1]]
+        ex |= np.abs(p32 - vk) <= EXEMPT_REL * abs(vk)
+        if kstar >= k_min:
+            amb = np.nonzero(np.abs(cs - g) <= EXEMPT_REL * g)[0]
+            for i in amb:
+                for j in (i - 1, i, i + 1, i + 2):
+                    if 0 <= j < nb:
+                        ex[order[j]] = True
+    return ex
+
+
+def pe_exempt(a_bar: np.ndarray, gamma: float) -> np.ndarray:
+    """Tiles of a PE head whose selection could flip under float rounding."""
+    nb = a_bar.shape[0]
+    ii, jj = np.tril_indices(nb)
+    vals = a_bar[ii, jj]
+    vals32 = (vals / vals.sum()).astype(np.float32)
+    flat = ii.astype(np.int64) * nb + jj
+    order = np.lexsort((flat, -vals32.astype(np.float64)))
+    cs = np.cumsum(vals32[order].astype(np.float64))
+    g = np.float64(np.float32(gamma))
+    hit = np.nonzero(cs >= g)[0]
+    ex = np.zeros((nb, nb), dtype=bool)
+    if not hit.size:
+        return ex
+    kstar = int(hit[0]) + 1
+    vk = vals32[order[kstar - 1]]
+    near = np.abs(vals32 - vk) <= EXEMPT_REL * abs(vk)
+    ex.flat[flat[near]] = True
+    amb = np.nonzero(np.abs(cs - g) <= EXEMPT_REL * g)[0]
+    for i in amb:
+        for j in (i - 1, i, i + 1, i + 2):
+            if 0 <= j < len(order):
+                ex.flat[flat[order[j]]] = True
+    return ex
+
+
+def compare_head(gpu, b, h, q_head, k_head, v_head, w, oprm, qblocks=None, score_tol=2e-5):
+    """Compares one query head; returns a report dict (asserts on hard failures)."""
+    bh = b * w.h_q + h
+    nb = w.n_blocks
+    rep = {"head": (b, h), "exempt_route": False, "exempt_blocks": 0}
+    orc = O.head_route_and_select(q_head, k_head, oprm)
+    gp = int(gpu["pattern"][bh])
+    # (1) block scores
+    np.testing.assert_allclose(gpu["p_v"][bh].double().numpy(), orc["p_v"], rtol=score_tol, atol=1e-9)
+    np.testing.assert_allclose(gpu["p_s"][bh].double().numpy(), orc["p_s"], rtol=score_tol, atol=1e-9)
+    # (2) route
+    tau = oprm.tau_jsd if oprm.router == "jsd" else oprm.tau_proxy
+    np.testing.assert_allclose(float(gpu["score"][bh]), orc["score"], rtol=score_tol, atol=1e-7)
+    if _near(orc["score"], tau):
+        rep["exempt_route"] = True
+        if gp != orc["routed"]:
+            orc = O.head_route_and_select(q_head, k_head, oprm, force_pattern=gp)
+    else:
+        assert gp == orc["routed"], (b, h, gp, orc["routed"], orc["score"])
+    rep["pattern"] = gp
+    gmask = gpu["mask"][bh].numpy().astype(bool)
+    # (3) selection
+    if gp == O.VS:
+        sel = gpu["vs_sel"][bh].numpy().astype(bool)
+        for d, (key, pd) in enumerate((("s_v", orc["p_v"]), ("s_s", orc["p_s"]))):
+            want = np.zeros(nb, dtype=bool)
+            want[orc[key]] = True
+            ex = vs_exempt(pd, oprm.vs_rule, oprm.alpha, oprm.gamma, oprm.k_min_blocks)
+            bad = (sel[d] != want) & ~ex
+            assert not bad.any(), (b, h, key, np.nonzero(bad)[0][:10])
+            rep["exempt_blocks"] += int(ex.sum())
+        s_v = np.nonzero(sel[0])[0]
+        s_s = np.nonzero(sel[1])[0]
+        np.testing.assert_array_equal(gmask, O.vs_tile_mask(s_v, s_s, nb))
+    else:
+        ex = pe_exempt(orc["a_bar"], oprm.gamma)
+        want = orc["mask"]
+        bad = (gmask != want) & ~ex
+        assert not bad.any(), (b, h, np.argwhere(bad)[:10])
+        idx = np.arange(nb)
+        assert gmask[idx, idx].all() and gmask[:, 0].all()
+        assert not np.triu(gmask, 1).any()
+        rep["exempt_blocks"] += int(ex.sum())
+    # (4) tile lists = ascending nonzeros of the mask row
+    cnt = gpu["tile_cnt"][bh].numpy()
+    np.testing.assert_array_equal(cnt, gmask.sum(axis=1))
+    tidx = gpu["tile_idx"][bh].numpy()
+    for qb in range(nb):
+        np.testing.assert_array_equal(tidx[qb, : cnt[qb]], np.nonzero(gmask[qb])[0])
+    rep["density"] = float(gmask.sum()) / (nb * (nb + 1) / 2)
+    # (5) attention on the GPU's own mask
+    o_ref, lse_ref, rows = O.masked_attention_rows(q_head, k_head, v_head, gmask, w.block,
+                                                   oprm.scale(q_head.shape[1]), qblocks)
+    o_gpu = gpu["o"][b, h].float().numpy()[rows]
+    lse_gpu = gpu["lse"][b, h].numpy()[rows]
+    err = np.abs(o_gpu - o_ref)
+    rep["attn_max_abs"] = float(err.max())
+    rep["attn_mean_abs"] = float(err.mean())
+    rep["attn_rel"] = float(err.max() / max(np.abs(o_ref).max(), 1e-30))
+    assert rep["attn_max_abs"] <= ATTN_MAX_ABS and rep["attn_mean_abs"] <= ATTN_MEAN_ABS, rep
+    np.testing.assert_allclose(lse_gpu, lse_ref, atol=2e-3, rtol=0)
+    return rep
+
+
+def sample_qblocks(nb: int, n_random: int, seed: int) -> Sequence[int]:
+    rng = np.random.default_rng(seed)
+    pick = {0, nb - 1}
+    pick.update(int(x) for x in rng.choice(np.arange(1, nb - 1), size=min(n_random, nb - 2), replace=False))
+    return sorted(pick)
+
+
+def compare_all(w, q, k, v, gpu, oprm, qblocks_fn=None, heads=None):
+    g = w.h_q // w.h_kv
+    reports = []
+    for b in range(w.batch):
+        for h in (range(w.h_q) if heads is None else heads):
+            qh = O.bf16_to_f64(q[b, h])
+            kh = O.bf16_to_f64(k[b, h // g])
+            vh = O.bf16_to_f64(v[b, h // g])
+            qbs = None if qblocks_fn is None else qblocks_fn(b, h)
+            reports.append(compare_head(gpu, b, h, qh, kh, vh, w, oprm, qbs))
+    return reports

@@ -1,0 +1,93 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/crisp.h declares, and rejects bad arguments with the
+documented status codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from dynamic_block_sparse_qk_b200 import binding as B
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "crisp.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(crisp_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from dynamic_block_sparse_qk_b200 import build
+    build.build()
+    return B.load_library()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared_functions()
+    assert set(names) == set(B.EXPORTED)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings(lib):
+    assert lib.crisp_version() == 10000
+    assert lib.crisp_status_string(0) == b"ok"
+    assert lib.crisp_status_string(-3) == b"workspace too small"
+
+
+def _p(**kw):
+    base = dict(batch=1, h_q=32, h_kv=8, seqlen=32768, head_dim=128, block=128)
+    base.update(kw)
+    return B.make_params(**base)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(h_q=30), -2), (dict(head_dim=96), -2), (dict(block=32), -2), (dict(seqlen=1000), -2),
+    (dict(seqlen=256), -2), (dict(seqlen=2 ** 21), -2), (dict(block=64, seqlen=2 ** 19), -2),
+    (dict(alpha=0.0), -1), (dict(gamma=1.5), -1), (dict(gamma=0.0), -1), (dict(k_min_blocks=0), -1),
+    (dict(router=7), -1), (dict(vs_rule=2), -1), (dict(sm_scale=-1.0), -1), (dict(batch=0), -2),
+    (dict(h_q=32, h_kv=0), -2),
+])
+def test_check_params_rejects(lib, kw, code):
+    p = _p(**kw)
+    assert lib.crisp_check_params(ctypes.byref(p)) == code
+    assert lib.crisp_workspace_size(ctypes.byref(p)) == 0
+
+
+def test_valid_configs_have_workspace(lib):
+    for kw in (dict(), dict(batch=1, h_q=2, h_kv=1, seqlen=2048, head_dim=64, block=64),
+               dict(h_q=28, h_kv=4, seqlen=131072), dict(seqlen=524288)):
+        p = _p(**kw)
+        assert lib.crisp_check_params(ctypes.byref(p)) == 0
+        assert lib.crisp_workspace_size(ctypes.byref(p)) > 0
+
+
+def test_entry_points_validate_before_launch(lib):
+    p = _p()
+    fake = ctypes.c_void_p(1 << 20)          # aligned, never dereferenced
+    need = lib.crisp_workspace_size(ctypes.byref(p))
+    # null / misaligned workspace, too-small workspace, null tensors
+    assert lib.crisp_route(ctypes.byref(p), fake, fake, None, need, fake, fake, fake, fake, None) == -1
+    assert lib.crisp_route(ctypes.byref(p), fake, fake, ctypes.c_void_p((1 << 20) + 8), need,
+                           fake, fake, fake, fake, None) == -1
+    assert lib.crisp_route(ctypes.byref(p), fake, fake, fake, need - 1, fake, fake, fake, fake, None) == -3
+    assert lib.crisp_route(ctypes.byref(p), None, fake, fake, need, fake, fake, fake, fake, None) == -1
+    assert lib.crisp_route(ctypes.byref(p), ctypes.c_void_p((1 << 20) + 2), fake, fake, need, fake,
+                           fake, fake, fake, None) == -1
+    assert lib.crisp_select(ctypes.byref(p), fake, fake, fake, fake, fake, fake, need, None, None,
+                            None, fake, None) == -1
+    assert lib.crisp_sparse_prefill(ctypes.byref(p), fake, fake, fake, fake, fake, None, None,
+                                    fake, need, None) == -1
+    assert lib.crisp_dense_prefill(ctypes.byref(p), fake, fake, None, fake, None, fake, need, None) == -1
+    bad = _p(block=96)
+    assert lib.crisp_dense_prefill(ctypes.byref(bad), fake, fake, fake, fake, None, fake, need, None) == -2
+    st = ctypes.c_int32(0)
+    assert lib.crisp_get_device_status(None, ctypes.byref(st), None) == -1
+
+
+def test_params_struct_layout_matches_header(lib):
+    # 10 int32 + 4 float fields, no padding
+    assert ctypes.sizeof(B.CrispParams) == 14 * 4

@@ -1,0 +1,152 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Routing and selected blocks are compared exactly outside the 1e-4 exemption
+band; attention against the oracle run on the GPU's own mask (max-abs 2e-2,
+mean-abs 2e-3). Larger configs sample query blocks for attention and check
+routing and selection in full.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from synthetic import WORKLOADS, Workload, make_qkv
+import parity_util as PU
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from dynamic_block_sparse_qk_b200 import build
+    build.build()
+
+
+def _check(w, router="cstruct", vs_rule="alpha", alpha=1.0, gamma=0.95, qblocks_fn=None,
+           heads=None, expect_both=False):
+    q, k, v, meta = make_qkv(w)
+    gpu = PU.run_gpu(w, q, k, v, router=router, vs_rule=vs_rule, alpha=alpha, gamma=gamma)
+    assert gpu["status"] == 0
+    oprm = PU.oracle_params(w, router=router, vs_rule=vs_rule, alpha=alpha, gamma=gamma)
+    reps = PU.compare_all(w, q, k, v, gpu, oprm, qblocks_fn=qblocks_fn, heads=heads)
+    if expect_both:
+        pats = {r["pattern"] for r in reps}
+        assert pats == {O.VS, O.PE}, pats
+    return reps
+
+
+@pytest.mark.parametrize("alpha", [0.5, 1.0, 2.0])
+def test_tiny_full(alpha):
+    reps = _check(WORKLOADS["tiny"], alpha=alpha, expect_both=True)
+    assert reps[0]["pattern"] == O.VS and reps[1]["pattern"] == O.PE
+
+
+def test_tiny_gamma_vs_rule():          # Abl.1: C_struct routing + gamma VS selection
+    _check(WORKLOADS["tiny"], vs_rule="gamma")
+
+
+def test_tiny_jsd_router():             # Abl.2: JSD routing + alpha VS selection
+    _check(WORKLOADS["tiny"], router="jsd")
+
+
+def test_tiny_unit_variance_values():   # V ~ N(0,1): the absolute tolerance bites
+    reps = _check(WORKLOADS["tiny"].with_(v_unit=True))
+    assert max(r["attn_max_abs"] for r in reps) < 2e-2
+
+
+@pytest.mark.parametrize("kw", [
+    dict(seqlen=384, block=128, head_dim=128, h_q=2, h_kv=1),              # N_b = 3 (smallest)
+    dict(seqlen=640, block=128, head_dim=64, h_q=4, h_kv=2),               # odd N_b, d=64 at B=128
+    dict(seqlen=1024, block=64, head_dim=128, h_q=3, h_kv=3),              # B=64 with d=128, g=1
+    dict(seqlen=1536, block=128, head_dim=128, h_q=4, h_kv=1, batch=2),    # batch 2, GQA g=4
+])
+def test_edge_shapes(kw):
+    base = dict(name="edge", batch=1, n_vertical=2, diffuse_frac=0.5, sink_logit=8.0)
+    base.update(kw)
+    _check(Workload(**base))
+
+
+def test_kmin_above_nb():
+    w = Workload("kmin", 1, 2, 1, 64, 512, 64, diffuse_heads=(1,), n_vertical=0, sink_logit=8.0)
+    q, k, v, _ = make_qkv(w)
+    import dynamic_block_sparse_qk_b200 as C
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    p = C.params_for(qd, kd, block=64, k_min_blocks=50)
+    ws = C.alloc_workspace(p)
+    pattern, score, pv, ps = C.crisp_route(p, qd, kd, ws)
+    mask, tidx, tcnt = C.crisp_select(p, qd, kd, pattern, pv, ps, ws)
+    if int(pattern[0]) == O.VS:      # k_min > N_b clips to N_b: every causal tile
+        assert torch.equal(mask[0].cpu().bool(), torch.tril(torch.ones(8, 8, dtype=torch.bool)))
+
+
+def test_dense_equals_oracle_full_mask():
+    w = Workload("dense", 1, 4, 2, 128, 1024, 128, n_vertical=2)
+    q, k, v, _ = make_qkv(w)
+    import dynamic_block_sparse_qk_b200 as C
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    p = C.params_for(qd, kd, block=128)
+    ws = C.alloc_workspace(p)
+    o, lse = C.crisp_dense_prefill(p, qd, kd, vd, ws)
+    assert C.crisp_get_device_status(ws) == 0
+    full = np.tril(np.ones((8, 8), dtype=bool))
+    for h in range(4):
+        ref, lref, rows = O.masked_attention_rows(O.bf16_to_f64(q[0, h]), O.bf16_to_f64(k[0, h // 2]),
+                                                  O.bf16_to_f64(v[0, h // 2]), full, 128, 128 ** -0.5)
+        err = np.abs(o[0, h].float().cpu().numpy() - ref)
+        assert err.max() <= 2e-2 and err.mean() <= 2e-3
+        np.testing.assert_allclose(lse[0, h].cpu().numpy(), lref, atol=2e-3)
+
+
+def test_sparse_with_full_lists_equals_dense():
+    w = Workload("full", 1, 2, 1, 128, 2048, 128)
+    q, k, v, _ = make_qkv(w)
+    import dynamic_block_sparse_qk_b200 as C
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    p = C.params_for(qd, kd, block=128)
+    ws = C.alloc_workspace(p)
+    nb = 16
+    tidx = torch.arange(nb, dtype=torch.int32, device="cuda").repeat(2, nb, 1).contiguous()
+    tcnt = torch.arange(1, nb + 1, dtype=torch.int32, device="cuda").repeat(2, 1).contiguous()
+    o1, l1 = C.crisp_sparse_prefill(p, qd, kd, vd, tidx, tcnt, ws)
+    o2, l2 = C.crisp_dense_prefill(p, qd, kd, vd, ws)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_out_of_range_tile_index_is_reported_not_read():
+    w = Workload("bad", 1, 1, 1, 128, 1024, 128, diffuse_heads=())
+    q, k, v, _ = make_qkv(w)
+    import dynamic_block_sparse_qk_b200 as C
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    p = C.params_for(qd, kd, block=128)
+    ws = C.alloc_workspace(p)
+    nb = 8
+    tidx = torch.zeros(1, nb, nb, dtype=torch.int32, device="cuda")
+    tidx[0, 3, 1] = 7            # key block 7 is above query block 3: rejected by the kernel
+    tcnt = torch.ones(1, nb, dtype=torch.int32, device="cuda")
+    tcnt[0, 3] = 2
+    C.crisp_sparse_prefill(p, qd, kd, vd, tidx, tcnt, ws)
+    assert C.crisp_get_device_status(ws) == -6
+    assert C.crisp_get_device_status(ws) == 0     # reading clears it
+
+
+def test_llama_32k():
+    w = WORKLOADS["llama_32k"]
+    reps = _check(w, qblocks_fn=lambda b, h: PU.sample_qblocks(w.n_blocks, 4, 1000 + h), expect_both=True)
+    vs = [r for r in reps if r["pattern"] == O.VS]
+    assert len(vs) == 24
+    assert max(r["density"] for r in vs) < 0.2
+
+
+@pytest.mark.slow
+def test_qwen_131k_alpha_and_gamma():
+    w = WORKLOADS["qwen_131k"]
+    for vs_rule in ("alpha", "gamma"):
+        _check(w, vs_rule=vs_rule, qblocks_fn=lambda b, h: PU.sample_qblocks(w.n_blocks, 2, 2000 + h))
+
+
+@pytest.mark.slow
+def test_llama_512k():
+    w = WORKLOADS["llama_512k"]
+    _check(w, qblocks_fn=lambda b, h: PU.sample_qblocks(w.n_blocks, 1, 3000 + h), expect_both=True)
