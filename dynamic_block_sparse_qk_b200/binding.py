@@ -25,7 +25,8 @@ PATTERN_VS, PATTERN_PE = 0, 1
 
 EXPORTED = ("crisp_version", "crisp_status_string", "crisp_check_params", "crisp_workspace_size",
             "crisp_route", "crisp_select", "crisp_sparse_prefill", "crisp_dense_prefill",
-            "crisp_get_device_status")
+            "crisp_get_device_status", "crisp_route_noalloc")
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class CrispError(RuntimeError):
@@ -89,6 +90,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.crisp_sparse_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.crisp_dense_prefill.restype = i32
     lib.crisp_dense_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.crisp_route_noalloc.restype = i32
+    lib.crisp_route_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
     lib.crisp_get_device_status.restype = i32
     lib.crisp_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), vp]
     _lib = lib
@@ -189,6 +192,26 @@ def crisp_dense_prefill(p: CrispParams, q, k, v, ws, o=None, lse=None, want_lse=
         ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(ws), ws.numel(),
         _stream(stream)))
     return o, lse
+
+
+def crisp_route_noalloc(p: CrispParams, q, k, pattern=None, score=None, p_v=None, p_s=None,
+                        stream=None):
+    """Routing for callers that may not allocate device memory: the same
+    kernels as crisp_route, with the library's fixed scratch array instead of
+    a workspace. Returns (pattern, score, p_v, p_s). Output tensors passed in
+    are used as given; when omitted they are created here by torch, which is
+    this wrapper's convenience, not the library's."""
+    _need_cuda(q, k)
+    bh, nb = p.batch * p.h_q, p.n_blocks
+    dev = q.device
+    pattern = torch.empty(bh, dtype=torch.int32, device=dev) if pattern is None else pattern
+    score = torch.empty(bh, dtype=torch.float32, device=dev) if score is None else score
+    p_v = torch.empty(bh, nb, dtype=torch.float32, device=dev) if p_v is None else p_v
+    p_s = torch.empty(bh, nb, dtype=torch.float32, device=dev) if p_s is None else p_s
+    _check("crisp_route_noalloc", load_library().crisp_route_noalloc(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(pattern), _ptr(score), _ptr(p_v), _ptr(p_s),
+        _stream(stream)))
+    return pattern, score, p_v, p_s
 
 
 def crisp_get_device_status(ws, stream=None) -> int:

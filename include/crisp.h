@@ -131,6 +131,26 @@ int crisp_sparse_prefill(const crisp_params* p, const void* q, const void* k, co
 int crisp_dense_prefill(const crisp_params* p, const void* q, const void* k, const void* v,
                         void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
 
+/* Routing without a caller workspace. The paper has no counterpart: this
+ * entry point exists for callers that may not allocate device memory — for
+ * example a plug-in whose host framework reserves all device memory for its
+ * own pool and passes no workspace, or a latency-critical loop that cannot
+ * take the device-wide synchronisation cudaMalloc may cause. It runs exactly
+ * the crisp_route kernels, with identical arguments and outputs minus the
+ * workspace, and calls no allocator. Its scratch is one fixed array of
+ * CRISP_NOALLOC_SCRATCH_BYTES in the library's device image, held by every
+ * GPU that loads the library until the process exits.
+ *  - Problems whose routing scratch exceeds that size (Llama shapes beyond
+ *    32k tokens, for instance) return CRISP_ERR_WORKSPACE without launching.
+ *  - All calls on a device share the array, which keeps the last call's
+ *    contents; calls whose kernels overlap on the GPU race. Issue them in
+ *    order on one stream.
+ *  - The first call on each device looks up the array's address (with that
+ *    device current); make that first call before any stream capture. */
+#define CRISP_NOALLOC_SCRATCH_BYTES (16u << 20)
+int crisp_route_noalloc(const crisp_params* p, const void* q, const void* k, int32_t* pattern,
+                        float* score, float* p_v, float* p_s, void* stream);
+
 /* Synchronises `stream`, copies the device status word out of `ws` into
  * *status (CRISP_OK or CRISP_ERR_TIMEOUT / CRISP_ERR_DEVICE) and clears it.
  * Returns CRISP_OK unless the copy itself failed. */
