@@ -43,6 +43,8 @@ int to_status(cudaError_t e) { return e == cudaSuccess ? CRISP_OK : CRISP_ERR_CU
 
 }  // namespace
 
+
+
 extern "C" {
 
 int crisp_version(void) { return 10000; }

@@ -1,0 +1,513 @@
+// Block-sparse causal GQA flash attention (CRISP paper, Eq. 1) on the
+// 5th-generation tensor cores of sm_100a.
+//
+// One CTA = one 128-row query tile of one head; it walks the 128-key tiles
+// that the tile lists select (the union over the query blocks the tile covers,
+// with a per-block membership mask), in ascending order.
+//
+//   warp 4 (one lane)  TMA producer: Q once, then K_j / V_j tiles into a ring
+//                      of shared-memory slots (128-byte swizzle).
+//   warp 5 (one lane)  UMMA issuer: S_j = Q K_j^T into one of two TMEM
+//                      buffers, then O += P_{j-1} V_{j-1} (O lives in TMEM),
+//                      so the QK^T of step j runs under the softmax of j-1.
+//   warps 0-3          softmax: thread r owns query row r (TMEM lane r):
+//                      tcgen05.ld of S, masking, online max with deferred
+//                      rescaling (O is rescaled in TMEM only when the row max
+//                      grows by more than 2^8), exp2, P written as bf16 into
+//                      a double-buffered swizzled shared tile that the PV
+//                      UMMA reads; final O / l and the log-sum-exp.
+//
+// Every mbarrier wait is bounded; a wait that runs out records
+// CRISP_ERR_TIMEOUT in the workspace status word and raises a CTA abort flag,
+// after which all roles leave their loops, the producer waits (bounded) for
+// its copies in flight and the TMEM allocation is released.
+#include <climits>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace crisp {
+using namespace sm100;
+
+namespace {
+
+constexpr int BM = 128;          // query rows per CTA (UMMA M)
+constexpr int BN = 128;          // keys per step (UMMA N of QK^T)
+constexpr int kThreads = 192;    // 4 softmax warps, 1 producer warp, 1 MMA warp
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct Cfg {
+  static constexpr int NSLOT = D == 128 ? 4 : 8;
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int P_BYTES = BM * BN * 2;
+  static constexpr int T_BYTES = BN * D * 2;          // one K or V tile
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_P = OFF_Q + Q_BYTES;
+  static constexpr int OFF_RING = OFF_P + 2 * P_BYTES;
+  static constexpr int OFF_BAR = OFF_RING + NSLOT * T_BYTES;
+  static constexpr int B_Q = 0, B_FULL = 1, B_EMPTY = 1 + NSLOT, B_S = 1 + 2 * NSLOT,
+                       B_P = B_S + 2, B_PV = B_P + 2, B_O = B_PV + 2, N_BARS = B_O + 1;
+  static constexpr int OFF_TMEM = OFF_BAR + 8 * N_BARS;
+  static constexpr int OFF_ABORT = OFF_TMEM + 8;
+  static constexpr int SMEM = OFF_ABORT + 8 + 1024;   // + alignment slack
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+// Walks the 128-key tiles a query tile needs, ascending, with membership bits:
+// bit (i * kpu + ks) says query block qb0+i attends key block kt*kpu+ks.
+struct StepIter {
+  const int32_t* lst[2];
+  int cnt[2], pos[2];
+  int nsub, kpu, qb0, dense_last, next_kt;
+  int32_t* status;
+  bool report;
+
+  __device__ void init(const int32_t* tile_idx, const int32_t* tile_cnt, int bh, int nb, int block,
+                       int qt, int32_t* st, bool rep) {
+    nsub = BM / block;
+    kpu = BN / block;
+    qb0 = qt * nsub;
+    status = st;
+    report = rep;
+    next_kt = 0;
+    dense_last = tile_idx ? -1 : qt;
+    for (int i = 0; i < 2; ++i) { lst[i] = nullptr; cnt[i] = 0; pos[i] = 0; }
+    if (tile_idx) {
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        if (i >= nsub) break;
+        const int qb = qb0 + i;
+        lst[i] = tile_idx + (size_t(bh) * nb + qb) * nb;
+        int c = tile_cnt[size_t(bh) * nb + qb];
+        if (c < 0 || c > qb + 1) {
+          if (report) report_error(status, CRISP_ERR_DEVICE, c);
+          c = c < 0 ? 0 : qb + 1;
+        }
+        cnt[i] = c;
+      }
+    }
+  }
+
+  __device__ bool next(int& kt, uint32_t& bits) {
+    if (dense_last >= 0) {
+      if (next_kt > dense_last) return false;
+      kt = next_kt++;
+      bits = 0;
+      for (int i = 0; i < nsub; ++i)
+        for (int ks = 0; ks < kpu; ++ks)
+          if (kt * kpu + ks <= qb0 + i) bits |= 1u << (i * kpu + ks);
+      return true;
+    }
+    int best = INT_MAX;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      if (i >= nsub) break;
+      while (pos[i] < cnt[i]) {
+        const int v = lst[i][pos[i]];
+        if (v >= 0 && v <= qb0 + i) break;
+        if (report) report_error(status, CRISP_ERR_DEVICE, v);
+        ++pos[i];
+      }
+      if (pos[i] < cnt[i]) best = min(best, lst[i][pos[i]] / kpu);
+    }
+    if (best == INT_MAX) return false;
+    bits = 0;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      if (i >= nsub) break;
+      while (pos[i] < cnt[i]) {
+        const int v = lst[i][pos[i]];
+        if (v < 0 || v > qb0 + i) {
+          if (report) report_error(status, CRISP_ERR_DEVICE, v);
+          ++pos[i];
+          continue;
+        }
+        if (v / kpu != best) break;
+        bits |= 1u << (i * kpu + v % kpu);
+        ++pos[i];
+      }
+    }
+    kt = best;
+    return true;
+  }
+};
+
+template <int D, int BLK>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                   const __grid_constant__ CUtensorMap tmv, const int32_t* __restrict__ tile_idx,
+                   const int32_t* __restrict__ tile_cnt, __nv_bfloat16* __restrict__ o,
+                   float* __restrict__ lse, crisp_params p, void* ws) {
+  using C = Cfg<D>;
+  constexpr int NSLOT = C::NSLOT;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* gbase = smem_raw + (base - raw);
+  const uint32_t sQ = base + C::OFF_Q, sP = base + C::OFF_P, sRing = base + C::OFF_RING;
+  auto BAR = [&](int i) -> uint32_t { return base + C::OFF_BAR + 8u * uint32_t(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_TMEM);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_ABORT);
+
+  const Workspace W = make_workspace(p);
+  int32_t* status = ws_ptr<int32_t>(ws, W.status);
+  const int N = p.seqlen, nb = N / p.block, NT = N / BM, BH = p.batch * p.h_q;
+  const int qt = NT - 1 - int(blockIdx.x) / BH;      // long rows first
+  const int bh = int(blockIdx.x) % BH;
+  const int b = bh / p.h_q, h = bh % p.h_q, hk = h / (p.h_q / p.h_kv);
+  const int row0 = qt * BM;
+  const int q_row = bh * N + row0;
+  const int kv_row0 = (b * p.h_kv + hk) * N;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(C::B_Q), 1);
+    for (int s = 0; s < NSLOT; ++s) {
+      mbar_init(BAR(C::B_FULL + s), 1);
+      mbar_init(BAR(C::B_EMPTY + s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(BAR(C::B_S + i), 1);
+      mbar_init(BAR(C::B_P + i), 4);     // one arrival per softmax warp
+      mbar_init(BAR(C::B_PV + i), 1);
+    }
+    mbar_init(BAR(C::B_O), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    prefetch_tmap(&tmq);
+    prefetch_tmap(&tmk);
+    prefetch_tmap(&tmv);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      StepIter it;
+      it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, true);
+      mbar_arrive_expect_tx(BAR(C::B_Q), C::Q_BYTES);
+      for (int box = 0; box < D / 64; ++box)
+        tma_load_2d(sQ + box * BM * 128, &tmq, box * 64, q_row, BAR(C::B_Q));
+      int t = 0;
+      auto load = [&](const CUtensorMap* m, int kt) -> bool {
+        const int s = t % NSLOT, u = t / NSLOT;
+        if (u >= 1 && !mbar_wait(BAR(C::B_EMPTY + s), (u - 1) & 1, abort_flag, status, 1)) return false;
+        mbar_arrive_expect_tx(BAR(C::B_FULL + s), C::T_BYTES);
+        for (int box = 0; box < D / 64; ++box)
+          tma_load_2d(sRing + s * C::T_BYTES + box * BN * 128, m, box * 64, kv_row0 + kt * BN,
+                      BAR(C::B_FULL + s));
+        ++t;
+        return true;
+      };
+      int kt, prev;
+      uint32_t bits;
+      if (it.next(kt, bits)) {
+        bool ok = load(&tmk, kt);
+        prev = kt;
+        while (ok && it.next(kt, bits)) {
+          ok = load(&tmk, kt) && load(&tmv, prev);
+          prev = kt;
+        }
+        if (ok) load(&tmv, prev);
+      }
+      // no copy may still be landing when the CTA exits
+      for (int s = 0; s < NSLOT && s < t; ++s) {
+        const int last = s + ((t - 1 - s) / NSLOT) * NSLOT;
+        if (!mbar_test(BAR(C::B_FULL + s), (last / NSLOT) & 1)) {
+          volatile int no_abort = 0;
+          mbar_wait(BAR(C::B_FULL + s), (last / NSLOT) & 1, &no_abort, status, 2, 1ll << 28);
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      StepIter it;
+      it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, false);
+      int n = 0, kt;
+      uint32_t bits;
+      while (it.next(kt, bits)) ++n;
+      constexpr uint32_t idq = idesc_bf16(BM, BN, 0);
+      constexpr uint32_t idp = idesc_bf16(BM, D, 1);
+      int t = 0;
+      auto wait_full = [&]() -> int {
+        const int s = t % NSLOT, u = t / NSLOT;
+        ++t;
+        return mbar_wait(BAR(C::B_FULL + s), u & 1, abort_flag, status, 3) ? s : -1;
+      };
+      auto issue_s = [&](int j, int s) {
+        const uint32_t d = tmem + uint32_t(j & 1) * 128u;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          const uint32_t boff = (kk >> 2) * (BN * 128) + (kk & 3) * 32;
+          umma_ss(d, smem_desc_sw128(sQ + aoff, 16, 1024),
+                  smem_desc_sw128(sRing + s * C::T_BYTES + boff, 16, 1024), idq, kk > 0);
+        }
+        umma_commit(BAR(C::B_S + (j & 1)));
+        umma_commit(BAR(C::B_EMPTY + s));
+      };
+      auto issue_pv = [&](int j, int s) {
+        const uint32_t d = tmem + 256u;
+        const uint32_t pb = sP + uint32_t(j & 1) * C::P_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          const uint32_t boff = kk * (16 * 128);
+          umma_ss(d, smem_desc_sw128(pb + aoff, 16, 1024),
+                  smem_desc_sw128(sRing + s * C::T_BYTES + boff, BN * 128, 1024), idp,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(BAR(C::B_PV + (j & 1)));
+        umma_commit(BAR(C::B_EMPTY + s));
+      };
+      bool ok = mbar_wait(BAR(C::B_Q), 0, abort_flag, status, 4);
+      if (ok && n > 0) {
+        int s = wait_full();
+        ok = s >= 0;
+        if (ok) { tc_fence_after(); issue_s(0, s); }
+        for (int j = 1; ok && j < n; ++j) {
+          s = wait_full();
+          ok = s >= 0;
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(j, s);
+          const int sv = wait_full();
+          ok = sv >= 0 && mbar_wait(BAR(C::B_P + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag, status, 5);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(j - 1, sv);
+        }
+        if (ok) {
+          const int sv = wait_full();
+          ok = sv >= 0 && mbar_wait(BAR(C::B_P + ((n - 1) & 1)), ((n - 1) >> 1) & 1, abort_flag, status, 6);
+          if (ok) {
+            tc_fence_after();
+            issue_pv(n - 1, sv);
+          }
+        }
+      }
+      umma_commit(BAR(C::B_O));
+    }
+  } else {
+    // ------------------------------------------------------------ softmax warps 0-3
+    const int r = threadIdx.x;                 // query row within the tile = TMEM lane
+    const int row = row0 + r;
+    const uint32_t lane_off = uint32_t(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_off, tO = tmem + lane_off + 256u;
+    constexpr int kpu = BN / BLK;
+    constexpr uint32_t kmask = (1u << kpu) - 1u;
+    const int qsub = r / BLK;
+    const float sl2 = (p.sm_scale > 0.f ? p.sm_scale : rsqrtf(float(D))) * kLog2e;
+    StepIter it;
+    it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, false);
+    float m_use = -INFINITY, l = 0.f;
+    int j = 0, kt;
+    uint32_t bits;
+    bool ok = true;
+    while (it.next(kt, bits)) {
+      ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_S + (j & 1)), (j >> 1) & 1, abort_flag, status, 7));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + uint32_t(j & 1) * 128u + c * 32, sr[c]);
+      tmem_wait_ld();
+      // Allowed key columns form one window [lo, hi]: the causal limit row - key0
+      // and, for 64-wide blocks, which halves of the key tile this row's query
+      // block selected.
+      const uint32_t rb = (bits >> (qsub * kpu)) & kmask;
+      const int lim = row - kt * BN;
+      int lo = 0, hi = lim < BN - 1 ? lim : BN - 1;
+      if (kpu == 2) {
+        if (!(rb & 1u)) lo = BLK;
+        if (!(rb & 2u)) hi = min(hi, BLK - 1);
+      } else if (!rb) {
+        hi = -1;
+      }
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (lo == 0 && hi == BN - 1) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float x = __uint_as_float(sr[c][e]) * sl2;
+            sr[c][e] = __float_as_uint(x);
+            mx[e & 3] = fmaxf(mx[e & 3], x);
+          }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int col = c * 32 + e;
+            const float x = (col >= lo && col <= hi) ? __uint_as_float(sr[c][e]) * sl2 : -INFINITY;
+            sr[c][e] = __float_as_uint(x);
+            mx[e & 3] = fmaxf(mx[e & 3], x);
+          }
+      }
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      float factor = 1.f;
+      bool resc = false;
+      if (j == 0) {
+        m_use = mt;
+      } else if (mt > m_use + 8.f) {
+        factor = fast_exp2(m_use - mt);
+        m_use = mt;
+        resc = true;
+      }
+      // the P buffer of step j was last read by PV_{j-2}
+      if (j >= 2) {
+        ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_PV + (j & 1)), ((j - 2) >> 1) & 1, abort_flag, status, 8));
+        if (!ok) break;
+      }
+      const uint32_t prow = sP + uint32_t(j & 1) * C::P_BYTES + uint32_t(r) * 128u;
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ch = 0; ch < 16; ++ch) {       // 16-byte chunk = 8 keys
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float a = fast_exp2(__uint_as_float(sr[ch >> 2][(ch & 3) * 8 + 2 * e]) - m_use);
+          const float bq = fast_exp2(__uint_as_float(sr[ch >> 2][(ch & 3) * 8 + 2 * e + 1]) - m_use);
+          rs[e] += a + bq;
+          pk[e] = pack_bf16(a, bq);
+        }
+        const uint32_t addr = prow + uint32_t(ch >> 3) * (BM * 128) + (uint32_t((ch & 7) ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]),
+                     "r"(pk[2]), "r"(pk[3])
+                     : "memory");
+      }
+      l = l * factor + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+      if (__any_sync(0xffffffffu, resc)) {
+        // O is final for step j-1 once PV_{j-1} completes; rescale it in TMEM
+        ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_PV + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag, status, 9));
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(tO + c * 32, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * factor);
+          tmem_st32(tO + c * 32, ov);
+        }
+        tmem_wait_st();
+      }
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::B_P + (j & 1)));
+      ++j;
+    }
+    __nv_bfloat16* orow = o + (size_t(bh) * N + row) * D;
+    const bool fin = ok && j > 0 &&
+                     __all_sync(0xffffffffu, mbar_wait(BAR(C::B_O), 0, abort_flag, status, 10));
+    if (fin) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        tmem_ld32(tO + c * 32, ov);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint4 u;
+          u.x = pack_bf16(__uint_as_float(ov[q4 * 8 + 0]) * inv, __uint_as_float(ov[q4 * 8 + 1]) * inv);
+          u.y = pack_bf16(__uint_as_float(ov[q4 * 8 + 2]) * inv, __uint_as_float(ov[q4 * 8 + 3]) * inv);
+          u.z = pack_bf16(__uint_as_float(ov[q4 * 8 + 4]) * inv, __uint_as_float(ov[q4 * 8 + 5]) * inv);
+          u.w = pack_bf16(__uint_as_float(ov[q4 * 8 + 6]) * inv, __uint_as_float(ov[q4 * 8 + 7]) * inv);
+          *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) = u;
+        }
+      }
+      if (lse) lse[size_t(bh) * N + row] = (m_use + log2f(l)) * kLn2;
+    } else {
+      for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+      if (lse) lse[size_t(bh) * N + row] = -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------------------------- host
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// Row-major [rows][d] bf16 matrix, 64-column x 128-row boxes, 128-byte swizzle.
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(d) * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int BLK>
+cudaError_t launch_tc(const crisp_params& p, const void* q, const void* k, const void* v,
+                      const int32_t* tile_idx, const int32_t* tile_cnt, void* o, float* lse, void* ws,
+                      cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  const uint64_t N = uint64_t(p.seqlen);
+  if (!make_tmap(&mq, q, uint64_t(p.batch) * p.h_q * N, D) || !make_tmap(&mk, k, uint64_t(p.batch) * p.h_kv * N, D) ||
+      !make_tmap(&mv, v, uint64_t(p.batch) * p.h_kv * N, D))
+    return cudaErrorInvalidValue;
+  auto kern = attn_tc_kernel<D, BLK>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = unsigned(p.batch) * p.h_q * (p.seqlen / BM);
+  kern<<<grid, kThreads, Cfg<D>::SMEM, st>>>(mq, mk, mv, tile_idx, tile_cnt, static_cast<__nv_bfloat16*>(o),
+                                             lse, p, ws);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t run_attention(const crisp_params& p, const void* q, const void* k, const void* v,
+                          const int32_t* tile_idx, const int32_t* tile_cnt, void* o, float* lse,
+                          void* ws, cudaStream_t st) {
+  if (p.head_dim == 64)
+    return p.block == 64 ? launch_tc<64, 64>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st)
+                         : launch_tc<64, 128>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st);
+  return p.block == 64 ? launch_tc<128, 64>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st)
+                       : launch_tc<128, 128>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st);
+}
+
+}  // namespace crisp

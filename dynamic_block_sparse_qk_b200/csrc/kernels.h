@@ -19,7 +19,7 @@ cudaError_t run_select(const crisp_params& p, const void* q, const void* k, cons
                        const float* p_v, const float* p_s, void* ws, uint8_t* mask,
                        int32_t* tile_idx, int32_t* tile_cnt, cudaStream_t st);
 
-// Block-sparse (tile_idx != NULL) or dense causal attention.
+// Block-sparse (tile_idx != NULL) or dense causal attention (tcgen05 kernel).
 cudaError_t run_attention(const crisp_params& p, const void* q, const void* k, const void* v,
                           const int32_t* tile_idx, const int32_t* tile_cnt, void* o, float* lse,
                           void* ws, cudaStream_t st);
