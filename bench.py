@@ -178,9 +178,10 @@ def run_ours(args, rank, world, local_rank):
 
     # dense baseline: same kernel, every causal tile (1 warm-up + args.dense_steps timed)
     od = torch.empty_like(q)
-    C.crisp_dense_prefill(p, q, k, v, ws, o=od, lse=lse, stream=stream)
-    torch.cuda.synchronize(dev)
     dts = []
+    if args.dense_steps > 0:
+        C.crisp_dense_prefill(p, q, k, v, ws, o=od, lse=lse, stream=stream)
+        torch.cuda.synchronize(dev)
     for _ in range(args.dense_steps):
         if flush is not None:
             flush.zero_()
@@ -190,7 +191,7 @@ def run_ours(args, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         dts.append(e0.elapsed_time(e1))
-    dense_ms = statistics.mean(dts)
+    dense_ms = statistics.mean(dts) if dts else float("nan")
     del od
 
     if world > 1:
