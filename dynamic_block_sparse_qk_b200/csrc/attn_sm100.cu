@@ -3,19 +3,25 @@
 //
 // One CTA = one 128-row query tile of one head; it walks the 128-key tiles
 // that the tile lists select (the union over the query blocks the tile covers,
-// with a per-block membership mask), in ascending order.
+// with a per-block membership mask), in ascending order: steps j = 0..n-1.
 //
-//   warp 4 (one lane)  TMA producer: Q once, then K_j / V_j tiles into a ring
-//                      of shared-memory slots (128-byte swizzle).
-//   warp 5 (one lane)  UMMA issuer: S_j = Q K_j^T into one of two TMEM
-//                      buffers, then O += P_{j-1} V_{j-1} (O lives in TMEM),
-//                      so the QK^T of step j runs under the softmax of j-1.
-//   warps 0-3          softmax: thread r owns query row r (TMEM lane r):
-//                      tcgen05.ld of S, masking, online max with deferred
-//                      rescaling (O is rescaled in TMEM only when the row max
-//                      grows by more than 2^8), exp2, P written as bf16 into
-//                      a double-buffered swizzled shared tile that the PV
-//                      UMMA reads; final O / l and the log-sum-exp.
+//   warp 8 (one lane)  TMA producer: Q once, then K and V tiles into a ring of
+//                      shared-memory slots (128-byte swizzle) in the order the
+//                      UMMAs consume them: K0, K1, then K_{j+2}, V_j per step.
+//   warp 9 (one lane)  UMMA issuer: S_j = Q K_j^T into TMEM buffer j%2 and
+//                      O_{j%2} += P_j V_j into one of two TMEM accumulators.
+//                      S_{j+2} is issued as soon as the softmax has read S_j.
+//   warps 0-3, 4-7     two softmax groups that ping-pong: group g takes the
+//                      steps j with j%2 == g, so one group's exp2 work overlaps
+//                      the other group's TMEM loads, stores and barriers.
+//                      Thread r of a group owns query row r (TMEM lane r):
+//                      tcgen05.ld of S, causal / block mask as one column
+//                      window, row max, exp2, P written as bf16 into its
+//                      group's swizzled shared tile for the PV UMMA; each group
+//                      keeps its own running max m_g and sum l_g and rescales
+//                      its accumulator in TMEM only when m_g grows by more
+//                      than 2^8. At the end the two partial results merge:
+//                      O = (O_0 2^(m_0-M) + O_1 2^(m_1-M)) / (l_0 2^(m_0-M) + l_1 2^(m_1-M)).
 //
 // Every mbarrier wait is bounded; a wait that runs out records
 // CRISP_ERR_TIMEOUT in the workspace status word and raises a CTA abort flag,
@@ -34,21 +40,23 @@ namespace {
 
 constexpr int BM = 128;          // query rows per CTA (UMMA M)
 constexpr int BN = 128;          // keys per step (UMMA N of QK^T)
-constexpr int kThreads = 192;    // 4 softmax warps, 1 producer warp, 1 MMA warp
-constexpr uint32_t kTmemCols = 512;
+constexpr int kThreads = 320;    // 2 x 4 softmax warps, 1 producer warp, 1 MMA warp
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;  // S_0, S_1 (128 each), O_0, O_1 (D each)
 
 template <int D>
 struct Cfg {
   static constexpr int NSLOT = D == 128 ? 4 : 8;
   static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int P_BYTES = BM * BN * 2;
-  static constexpr int T_BYTES = BN * D * 2;          // one K or V tile
+  static constexpr int P_BYTES = BM * BN * 2;          // one group's P tile
+  static constexpr int T_BYTES = BN * D * 2;           // one K or V tile
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_P = OFF_Q + Q_BYTES;
   static constexpr int OFF_RING = OFF_P + 2 * P_BYTES;
   static constexpr int OFF_BAR = OFF_RING + NSLOT * T_BYTES;
   static constexpr int B_Q = 0, B_FULL = 1, B_EMPTY = 1 + NSLOT, B_S = 1 + 2 * NSLOT,
-                       B_P = B_S + 2, B_PV = B_P + 2, B_O = B_PV + 2, N_BARS = B_O + 1;
+                       B_SFREE = B_S + 2, B_P = B_SFREE + 2, B_PV = B_P + 2, B_O = B_PV + 2,
+                       N_BARS = B_O + 1;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * N_BARS;
   static constexpr int OFF_ABORT = OFF_TMEM + 8;
   static constexpr int SMEM = OFF_ABORT + 8 + 1024;   // + alignment slack
@@ -168,20 +176,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(BAR(C::B_FULL + s), 1);
       mbar_init(BAR(C::B_EMPTY + s), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(BAR(C::B_S + i), 1);
-      mbar_init(BAR(C::B_P + i), 4);     // one arrival per softmax warp
-      mbar_init(BAR(C::B_PV + i), 1);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(BAR(C::B_S + g), 1);
+      mbar_init(BAR(C::B_SFREE + g), 4);   // one arrival per warp of group g
+      mbar_init(BAR(C::B_P + g), 4);
+      mbar_init(BAR(C::B_PV + g), 1);
     }
     mbar_init(BAR(C::B_O), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&tmq);
     prefetch_tmap(&tmk);
     prefetch_tmap(&tmv);
@@ -191,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       StepIter it;
@@ -210,16 +219,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++t;
         return true;
       };
-      int kt, prev;
+      // key tiles of steps j, j+1, j+2 (the iterator runs two steps ahead)
+      int ktr[4] = {0, 0, 0, 0};
       uint32_t bits;
-      if (it.next(kt, bits)) {
-        bool ok = load(&tmk, kt);
-        prev = kt;
-        while (ok && it.next(kt, bits)) {
-          ok = load(&tmk, kt) && load(&tmv, prev);
-          prev = kt;
+      int have = 0;
+      while (have < 2 && it.next(ktr[have], bits)) ++have;
+      bool ok = true;
+      for (int i = 0; i < have && ok; ++i) ok = load(&tmk, ktr[i]);
+      for (int j = 0; ok && j < have; ++j) {
+        int kt2;
+        if (it.next(kt2, bits)) {
+          ktr[(j + 2) & 3] = kt2;
+          ++have;
+          ok = load(&tmk, kt2);
         }
-        if (ok) load(&tmv, prev);
+        if (ok) ok = load(&tmv, ktr[j & 3]);
       }
       // no copy may still be landing when the CTA exits
       for (int s = 0; s < NSLOT && s < t; ++s) {
@@ -230,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
       StepIter it;
@@ -259,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(BAR(C::B_EMPTY + s));
       };
       auto issue_pv = [&](int j, int s) {
-        const uint32_t d = tmem + 256u;
+        const uint32_t d = tmem + 256u + uint32_t(j & 1) * D;
         const uint32_t pb = sP + uint32_t(j & 1) * C::P_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
@@ -267,45 +281,46 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t boff = kk * (16 * 128);
           umma_ss(d, smem_desc_sw128(pb + aoff, 16, 1024),
                   smem_desc_sw128(sRing + s * C::T_BYTES + boff, BN * 128, 1024), idp,
-                  (j > 0 || kk > 0) ? 1u : 0u);
+                  (j >= 2 || kk > 0) ? 1u : 0u);
         }
         umma_commit(BAR(C::B_PV + (j & 1)));
         umma_commit(BAR(C::B_EMPTY + s));
       };
       bool ok = mbar_wait(BAR(C::B_Q), 0, abort_flag, status, 4);
-      if (ok && n > 0) {
-        int s = wait_full();
+      for (int j = 0; ok && j < 2 && j < n; ++j) {
+        const int s = wait_full();
         ok = s >= 0;
-        if (ok) { tc_fence_after(); issue_s(0, s); }
-        for (int j = 1; ok && j < n; ++j) {
-          s = wait_full();
+        if (ok) { tc_fence_after(); issue_s(j, s); }
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        if (j + 2 < n) {
+          // S buffer j%2 is free once its softmax group has read S_j
+          ok = mbar_wait(BAR(C::B_SFREE + (j & 1)), (j >> 1) & 1, abort_flag, status, 5);
+          if (!ok) break;
+          const int s = wait_full();
           ok = s >= 0;
           if (!ok) break;
           tc_fence_after();
-          issue_s(j, s);
-          const int sv = wait_full();
-          ok = sv >= 0 && mbar_wait(BAR(C::B_P + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag, status, 5);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(j - 1, sv);
+          issue_s(j + 2, s);
         }
-        if (ok) {
-          const int sv = wait_full();
-          ok = sv >= 0 && mbar_wait(BAR(C::B_P + ((n - 1) & 1)), ((n - 1) >> 1) & 1, abort_flag, status, 6);
-          if (ok) {
-            tc_fence_after();
-            issue_pv(n - 1, sv);
-          }
-        }
+        const int sv = wait_full();
+        ok = sv >= 0 && mbar_wait(BAR(C::B_P + (j & 1)), (j >> 1) & 1, abort_flag, status, 6);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(j, sv);
       }
       umma_commit(BAR(C::B_O));
     }
   } else {
-    // ------------------------------------------------------------ softmax warps 0-3
-    const int r = threadIdx.x;                 // query row within the tile = TMEM lane
+    // ------------------------------------------------------------ softmax groups
+    const int grp = warp >> 2, quad = warp & 3;
+    const int r = quad * 32 + lane;               // query row within the tile = TMEM lane
     const int row = row0 + r;
-    const uint32_t lane_off = uint32_t(warp * 32) << 16;
-    const uint32_t tS = tmem + lane_off, tO = tmem + lane_off + 256u;
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off + uint32_t(grp) * 128u;
+    const uint32_t tO0 = tmem + lane_off + 256u;  // O_0; O_1 at + D
+    const uint32_t tO = tO0 + uint32_t(grp) * D;
+    const uint32_t prow = sP + uint32_t(grp) * C::P_BYTES + uint32_t(r) * 128u;
     constexpr int kpu = BN / BLK;
     constexpr uint32_t kmask = (1u << kpu) - 1u;
     const int qsub = r / BLK;
@@ -313,17 +328,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     StepIter it;
     it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, false);
     float m_use = -INFINITY, l = 0.f;
-    int j = 0, kt;
+    int j = 0, u = 0, kt;
     uint32_t bits;
     bool ok = true;
     while (it.next(kt, bits)) {
-      ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_S + (j & 1)), (j >> 1) & 1, abort_flag, status, 7));
+      if ((j & 1) != grp) { ++j; continue; }
+      ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_S + grp), u & 1, abort_flag, status, 7));
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + uint32_t(j & 1) * 128u + c * 32, sr[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
       tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::B_SFREE + grp));      // S buffer may be overwritten
       // Allowed key columns form one window [lo, hi]: the causal limit row - key0
       // and, for 64-wide blocks, which halves of the key tile this row's query
       // block selected.
@@ -341,48 +360,44 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float x = __uint_as_float(sr[c][e]) * sl2;
-            sr[c][e] = __float_as_uint(x);
-            mx[e & 3] = fmaxf(mx[e & 3], x);
-          }
+          for (int e = 0; e < 32; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(sr[c][e]));
       } else {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int col = c * 32 + e;
-            const float x = (col >= lo && col <= hi) ? __uint_as_float(sr[c][e]) * sl2 : -INFINITY;
+            const float x = (col >= lo && col <= hi) ? __uint_as_float(sr[c][e]) : -INFINITY;
             sr[c][e] = __float_as_uint(x);
             mx[e & 3] = fmaxf(mx[e & 3], x);
           }
       }
-      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * sl2;
       float factor = 1.f;
       bool resc = false;
-      if (j == 0) {
-        m_use = mt;
+      if (u == 0) {
+        m_use = mt;                      // the first step of either group has a visible key
       } else if (mt > m_use + 8.f) {
         factor = fast_exp2(m_use - mt);
         m_use = mt;
         resc = true;
       }
-      // the P buffer of step j was last read by PV_{j-2}
-      if (j >= 2) {
-        ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_PV + (j & 1)), ((j - 2) >> 1) & 1, abort_flag, status, 8));
+      const float mref = m_use == -INFINITY ? 0.f : m_use;
+      // this group's P tile and O accumulator are free once its PV of step j-2 completed
+      if (u >= 1) {
+        ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_PV + grp), (u - 1) & 1, abort_flag, status, 8));
         if (!ok) break;
       }
-      const uint32_t prow = sP + uint32_t(j & 1) * C::P_BYTES + uint32_t(r) * 128u;
       float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {       // 16-byte chunk = 8 keys
+      for (int ch = 0; ch < 16; ++ch) {          // 16-byte chunk = 8 keys
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float a = fast_exp2(__uint_as_float(sr[ch >> 2][(ch & 3) * 8 + 2 * e]) - m_use);
-          const float bq = fast_exp2(__uint_as_float(sr[ch >> 2][(ch & 3) * 8 + 2 * e + 1]) - m_use);
+          const float a = fast_exp2(fmaf(__uint_as_float(sr[ch >> 2][(ch & 3) * 8 + 2 * e]), sl2, -mref));
+          const float bq = fast_exp2(fmaf(__uint_as_float(sr[ch >> 2][(ch & 3) * 8 + 2 * e + 1]), sl2, -mref));
           rs[e] += a + bq;
-          pk[e] = pack_bf16(a, bq);
+          pk[e] = pack_bf16_alu(a, bq);
         }
         const uint32_t addr = prow + uint32_t(ch >> 3) * (BM * 128) + (uint32_t((ch & 7) ^ (r & 7)) << 4);
         asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]),
@@ -391,9 +406,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       l = l * factor + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
       if (__any_sync(0xffffffffu, resc)) {
-        // O is final for step j-1 once PV_{j-1} completes; rescale it in TMEM
-        ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_PV + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag, status, 9));
-        if (!ok) break;
         tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
@@ -409,40 +421,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(C::B_P + (j & 1)));
+      if (lane == 0) mbar_arrive(BAR(C::B_P + grp));
       ++j;
+      ++u;
     }
-    __nv_bfloat16* orow = o + (size_t(bh) * N + row) * D;
-    const bool fin = ok && j > 0 &&
-                     __all_sync(0xffffffffu, mbar_wait(BAR(C::B_O), 0, abort_flag, status, 10));
+    // ---- merge the two groups' partial results (every softmax thread gets here once)
+    const bool done = ok && __all_sync(0xffffffffu, mbar_wait(BAR(C::B_O), 0, abort_flag, status, 10));
+    // all UMMAs have completed: the P tiles are free and hold the exchange
+    float* xch = reinterpret_cast<float*>(gbase + C::OFF_P);
+    xch[grp * 256 + r] = done ? m_use : -INFINITY;
+    xch[grp * 256 + 128 + r] = done ? l : 0.f;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    const float m0 = xch[r], l0 = xch[128 + r], m1 = xch[256 + r], l1 = xch[384 + r];
+    const float mm = fmaxf(m0, m1);
+    const float w0 = l0 > 0.f ? fast_exp2(m0 - mm) : 0.f;
+    const float w1 = l1 > 0.f ? fast_exp2(m1 - mm) : 0.f;
+    const float lt = l0 * w0 + l1 * w1;
+    __nv_bfloat16* orow = o + (size_t(bh) * N + row) * D + grp * (D / 2);
+    const bool fin = __all_sync(0xffffffffu, done && lt > 0.f);
     if (fin) {
       tc_fence_after();
-      const float inv = 1.f / l;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t ov[32];
-        tmem_ld32(tO + c * 32, ov);
+      const float a0 = w0 / lt, a1 = w1 / lt;
+#pragma unroll 1
+      for (int c = 0; c < D / 64; ++c) {
+        const uint32_t col = uint32_t(grp) * (D / 2) + c * 32;
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tO0 + col, v0);
+        tmem_ld32(tO0 + D + col, v1);
         tmem_wait_ld();
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          uint4 u;
-          u.x = pack_bf16(__uint_as_float(ov[q4 * 8 + 0]) * inv, __uint_as_float(ov[q4 * 8 + 1]) * inv);
-          u.y = pack_bf16(__uint_as_float(ov[q4 * 8 + 2]) * inv, __uint_as_float(ov[q4 * 8 + 3]) * inv);
-          u.z = pack_bf16(__uint_as_float(ov[q4 * 8 + 4]) * inv, __uint_as_float(ov[q4 * 8 + 5]) * inv);
-          u.w = pack_bf16(__uint_as_float(ov[q4 * 8 + 6]) * inv, __uint_as_float(ov[q4 * 8 + 7]) * inv);
-          *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) = u;
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float x0 = a0 != 0.f ? __uint_as_float(v0[q4 * 8 + e]) * a0 : 0.f;
+            const float x1 = a1 != 0.f ? __uint_as_float(v1[q4 * 8 + e]) * a1 : 0.f;
+            f[e] = x0 + x1;
+          }
+          uint4 pk;
+          pk.x = pack_bf16(f[0], f[1]);
+          pk.y = pack_bf16(f[2], f[3]);
+          pk.z = pack_bf16(f[4], f[5]);
+          pk.w = pack_bf16(f[6], f[7]);
+          *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) = pk;
         }
       }
-      if (lse) lse[size_t(bh) * N + row] = (m_use + log2f(l)) * kLn2;
+      if (lse && grp == 0) lse[size_t(bh) * N + row] = (mm + log2f(lt)) * kLn2;
     } else {
-      for (int c = 0; c < D; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
-      if (lse) lse[size_t(bh) * N + row] = -INFINITY;
+      for (int c = 0; c < D / 2; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
+      if (lse && grp == 0) lse[size_t(bh) * N + row] = -INFINITY;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);

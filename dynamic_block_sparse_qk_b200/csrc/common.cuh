@@ -156,6 +156,17 @@ __device__ inline uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// bf16x2 packing on the integer pipes (keeps the transcendental unit free for
+// exp2): round half up in the 16 dropped bits, then take both high halves with
+// one byte permute. For finite non-negative inputs this differs from
+// round-to-nearest-even only on exact ties.
+__device__ inline uint32_t pack_bf16_alu(float lo, float hi) {
+  const uint32_t a = __float_as_uint(lo) + 0x8000u, b = __float_as_uint(hi) + 0x8000u;
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // Byte offset of 16-byte chunk `chunk` of row `row` in a tile whose rows are
 // `row_bytes` long, with the chunk index XOR-swizzled by (row % 8).
 __device__ inline uint32_t swz(int row, int chunk, int row_bytes) {
