@@ -102,6 +102,19 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def max_over_ranks(values, device):
+    """Element-wise max of a list of floats over all ranks (identity when not
+    distributed). Each rank times its own replica; the job's time is the
+    slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(x) for x in values]
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 def launches_per_step(router: str) -> dict:
     """Kernels of this library launched by one call of each stage."""
     route = 4 + (1 if router == "jsd" else 0)      # proxy stats, merge, scores, (K pool), route
@@ -194,12 +207,7 @@ def run_ours(args, rank, world, local_rank):
     dense_ms = statistics.mean(dts) if dts else float("nan")
     del od
 
-    if world > 1:
-        t = torch.tensor([ms_local, dense_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, dense_ms = float(t[0]), float(t[1])
-    else:
-        ms = ms_local
+    ms, dense_ms = max_over_ranks([ms_local, dense_ms], dev)
 
     # end-to-end through the public API with host buffers (H2D inputs, D2H output)
     e2e = None
@@ -230,11 +238,7 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = e0.elapsed_time(e1) / args.steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t[0])
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], dev)[0]
         e2e = {"value": round(e2e_ms, 3), "unit": "ms",
                "h2d_bytes_per_step": int(in_bytes), "d2h_bytes_per_step": int(o.numel() * o.element_size())}
         del hq, hk, hv, ho
@@ -273,6 +277,98 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk.summary(),
     }
     return line
+
+
+# ----------------------------------------------------------------------------- sweep
+SWEEP_N = (8192, 16384, 32768, 65536, 131072, 262144, 524288)
+SWEEP_F = (0.0, 0.25, 0.5)
+SWEEP_ALPHA = (0.5, 1.0, 2.0)
+
+
+def run_sweep(args, out_path):
+    """Llama-shaped sweep: sequence length x diffuse-head fraction x alpha.
+
+    One JSON line per point: per-stage ms (route, select, attend), dense ms
+    (same kernel, every causal tile, once per (N, f)), speedup, selected-tile
+    density and the agreement of the C_struct and JSD routers on the heads.
+    Points already present in out_path are skipped, so an interrupted sweep
+    resumes where it stopped."""
+    import torch
+    import dynamic_block_sparse_qk_b200 as C
+    from synthetic import make_qkv, sweep_workload
+
+    done = set()
+    if os.path.exists(out_path):
+        with open(out_path) as f:
+            for line in f:
+                try:
+                    d = json.loads(line)
+                    done.add((d["seq_len"], d["diffuse_frac"], d["alpha"]))
+                except (ValueError, KeyError):
+                    pass
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    reps = max(1, args.steps)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / reps
+
+    for n in SWEEP_N:
+        for f in SWEEP_F:
+            todo = [a for a in SWEEP_ALPHA if (n, f, a) not in done]
+            if not todo:
+                continue
+            w = sweep_workload(n, f).with_(seed=args.seed)
+            q, k, v, _ = make_qkv(w, device=str(dev))
+            base = C.params_for(q, k, block=w.block)
+            ws = C.alloc_workspace(base, dev)
+            dense_ms = timed(lambda: C.crisp_dense_prefill(base, q, k, v, ws))
+            pj = C.params_for(q, k, block=w.block, router="jsd")
+            pat_j = C.crisp_route(pj, q, k, ws)[0].clone()
+            for a in todo:
+                p = C.params_for(q, k, block=w.block, alpha=a)
+                out = {}
+
+                def route():
+                    out["r"] = C.crisp_route(p, q, k, ws)
+
+                def select():
+                    r = out["r"]
+                    out["s"] = C.crisp_select(p, q, k, r[0], r[2], r[3], ws, want_mask=False)
+
+                def attend():
+                    s = out["s"]
+                    out["a"] = C.crisp_sparse_prefill(p, q, k, v, s[1], s[2], ws, want_lse=False)
+
+                t_route = timed(route)
+                t_select = timed(select)
+                t_attend = timed(attend)
+                pattern, tcnt = out["r"][0], out["s"][2]
+                nb = w.n_blocks
+                causal = p.batch * p.h_q * nb * (nb + 1) // 2
+                total = t_route + t_select + t_attend
+                rec = {"seq_len": n, "diffuse_frac": f, "alpha": a, "workload": w.name,
+                       "route_ms": round(t_route, 4), "select_ms": round(t_select, 4),
+                       "attend_ms": round(t_attend, 4), "total_ms": round(total, 4),
+                       "dense_ms": round(dense_ms, 4), "speedup_vs_dense": round(dense_ms / total, 3),
+                       "density": round(int(tcnt.sum()) / causal, 5),
+                       "vs_heads": int((pattern == 0).sum()), "heads": p.batch * p.h_q,
+                       "cstruct_jsd_agreement": round(float((pattern == pat_j).float().mean()), 4),
+                       "attend_tflops": round(int(tcnt.sum()) * 4 * w.block ** 2 * w.head_dim
+                                              / (t_attend * 1e-3) / 1e12, 1)}
+                with open(out_path, "a") as fo:
+                    fo.write(json.dumps(rec) + "\n")
+                print(json.dumps(rec), flush=True)
+            del q, k, v, ws
+            torch.cuda.empty_cache()
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -370,7 +466,11 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--sweep", default=None, help="write the N x f x alpha sweep to this JSONL file")
     args = ap.parse_args()
+    if args.sweep:
+        run_sweep(args, args.sweep)
+        return
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))

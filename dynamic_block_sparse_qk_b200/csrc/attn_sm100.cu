@@ -5,12 +5,14 @@
 // that the tile lists select (the union over the query blocks the tile covers,
 // with a per-block membership mask), in ascending order: steps j = 0..n-1.
 //
-//   warp 8 (one lane)  TMA producer: Q once, then K and V tiles into a ring of
-//                      shared-memory slots (128-byte swizzle) in the order the
-//                      UMMAs consume them: K0, K1, then K_{j+2}, V_j per step.
-//   warp 9 (one lane)  UMMA issuer: S_j = Q K_j^T into TMEM buffer j%2 and
-//                      O_{j%2} += P_j V_j into one of two TMEM accumulators.
-//                      S_{j+2} is issued as soon as the softmax has read S_j.
+//   warp 8 (one lane)  TMA producer of Q and of the K tiles (two-slot ring).
+//   warp 10 (one lane) TMA producer of the V tiles (two-slot ring).
+//   warp 9 (one lane)  UMMA issuer of S_j = Q K_j^T into TMEM buffer j%2, as
+//                      soon as the softmax has read S_{j-2} from that buffer.
+//   warp 11 (one lane) UMMA issuer of O_{j%2} += P_j V_j into one of two TMEM
+//                      accumulators, as soon as P_j is written. The two issuers
+//                      touch disjoint buffers, so a late V tile never holds up
+//                      the next QK^T and vice versa.
 //   warps 0-3, 4-7     two softmax groups that ping-pong: group g takes the
 //                      steps j with j%2 == g, so one group's exp2 work overlaps
 //                      the other group's TMEM loads, stores and barriers.
@@ -40,23 +42,24 @@ namespace {
 
 constexpr int BM = 128;          // query rows per CTA (UMMA M)
 constexpr int BN = 128;          // keys per step (UMMA N of QK^T)
-constexpr int kThreads = 320;    // 2 x 4 softmax warps, 1 producer warp, 1 MMA warp
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = 384;    // 2 x 4 softmax warps, 2 producer warps, 2 UMMA warps
+constexpr int kKProdWarp = 8, kSWarp = 9, kVProdWarp = 10, kPVWarp = 11;
 constexpr uint32_t kTmemCols = 512;  // S_0, S_1 (128 each), O_0, O_1 (D each)
 
 template <int D>
 struct Cfg {
-  static constexpr int NSLOT = D == 128 ? 4 : 8;
+  static constexpr int NSLOT = D == 128 ? 2 : 4;          // per ring (K and V)
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int P_BYTES = BM * BN * 2;          // one group's P tile
   static constexpr int T_BYTES = BN * D * 2;           // one K or V tile
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_P = OFF_Q + Q_BYTES;
   static constexpr int OFF_RING = OFF_P + 2 * P_BYTES;
-  static constexpr int OFF_BAR = OFF_RING + NSLOT * T_BYTES;
-  static constexpr int B_Q = 0, B_FULL = 1, B_EMPTY = 1 + NSLOT, B_S = 1 + 2 * NSLOT,
-                       B_SFREE = B_S + 2, B_P = B_SFREE + 2, B_PV = B_P + 2, B_O = B_PV + 2,
-                       N_BARS = B_O + 1;
+  static constexpr int OFF_VRING = OFF_RING + NSLOT * T_BYTES;
+  static constexpr int OFF_BAR = OFF_VRING + NSLOT * T_BYTES;
+  static constexpr int B_Q = 0, B_KFULL = 1, B_KEMPTY = 1 + NSLOT, B_VFULL = 1 + 2 * NSLOT,
+                       B_VEMPTY = 1 + 3 * NSLOT, B_S = 1 + 4 * NSLOT, B_SFREE = B_S + 2,
+                       B_P = B_SFREE + 2, B_PV = B_P + 2, B_O = B_PV + 2, N_BARS = B_O + 1;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * N_BARS;
   static constexpr int OFF_ABORT = OFF_TMEM + 8;
   static constexpr int SMEM = OFF_ABORT + 8 + 1024;   // + alignment slack
@@ -155,6 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   unsigned char* gbase = smem_raw + (base - raw);
   const uint32_t sQ = base + C::OFF_Q, sP = base + C::OFF_P, sRing = base + C::OFF_RING;
+  const uint32_t sVRing = base + C::OFF_VRING;
   auto BAR = [&](int i) -> uint32_t { return base + C::OFF_BAR + 8u * uint32_t(i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_TMEM);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_ABORT);
@@ -173,8 +177,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(BAR(C::B_Q), 1);
     for (int s = 0; s < NSLOT; ++s) {
-      mbar_init(BAR(C::B_FULL + s), 1);
-      mbar_init(BAR(C::B_EMPTY + s), 1);
+      mbar_init(BAR(C::B_KFULL + s), 1);
+      mbar_init(BAR(C::B_KEMPTY + s), 1);
+      mbar_init(BAR(C::B_VFULL + s), 1);
+      mbar_init(BAR(C::B_VEMPTY + s), 1);
     }
     for (int g = 0; g < 2; ++g) {
       mbar_init(BAR(C::B_S + g), 1);
@@ -186,11 +192,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == kSWarp) {
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
-  if (warp == kProducerWarp && lane == 0) {
+  if (warp == kKProdWarp && lane == 0) {
     prefetch_tmap(&tmq);
     prefetch_tmap(&tmk);
     prefetch_tmap(&tmv);
@@ -200,67 +206,57 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == kKProdWarp || warp == kVProdWarp) {
+    // ------------------------------------------------------------ TMA producers
     if (lane == 0) {
+      const bool is_k = warp == kKProdWarp;
+      const CUtensorMap* map = is_k ? &tmk : &tmv;
+      const uint32_t ring = is_k ? sRing : sVRing;
+      const int bfull = is_k ? C::B_KFULL : C::B_VFULL, bempty = is_k ? C::B_KEMPTY : C::B_VEMPTY;
       StepIter it;
-      it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, true);
-      mbar_arrive_expect_tx(BAR(C::B_Q), C::Q_BYTES);
-      for (int box = 0; box < D / 64; ++box)
-        tma_load_2d(sQ + box * BM * 128, &tmq, box * 64, q_row, BAR(C::B_Q));
-      int t = 0;
-      auto load = [&](const CUtensorMap* m, int kt) -> bool {
-        const int s = t % NSLOT, u = t / NSLOT;
-        if (u >= 1 && !mbar_wait(BAR(C::B_EMPTY + s), (u - 1) & 1, abort_flag, status, 1)) return false;
-        mbar_arrive_expect_tx(BAR(C::B_FULL + s), C::T_BYTES);
+      it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, is_k);
+      if (is_k) {
+        mbar_arrive_expect_tx(BAR(C::B_Q), C::Q_BYTES);
         for (int box = 0; box < D / 64; ++box)
-          tma_load_2d(sRing + s * C::T_BYTES + box * BN * 128, m, box * 64, kv_row0 + kt * BN,
-                      BAR(C::B_FULL + s));
-        ++t;
-        return true;
-      };
-      // key tiles of steps j, j+1, j+2 (the iterator runs two steps ahead)
-      int ktr[4] = {0, 0, 0, 0};
+          tma_load_2d(sQ + box * BM * 128, &tmq, box * 64, q_row, BAR(C::B_Q));
+      }
+      int t = 0, kt;
       uint32_t bits;
-      int have = 0;
-      while (have < 2 && it.next(ktr[have], bits)) ++have;
-      bool ok = true;
-      for (int i = 0; i < have && ok; ++i) ok = load(&tmk, ktr[i]);
-      for (int j = 0; ok && j < have; ++j) {
-        int kt2;
-        if (it.next(kt2, bits)) {
-          ktr[(j + 2) & 3] = kt2;
-          ++have;
-          ok = load(&tmk, kt2);
-        }
-        if (ok) ok = load(&tmv, ktr[j & 3]);
+      while (it.next(kt, bits)) {
+        const int s = t % NSLOT, u = t / NSLOT;
+        if (u >= 1 && !mbar_wait(BAR(bempty + s), (u - 1) & 1, abort_flag, status, 1)) break;
+        mbar_arrive_expect_tx(BAR(bfull + s), C::T_BYTES);
+        for (int box = 0; box < D / 64; ++box)
+          tma_load_2d(ring + s * C::T_BYTES + box * BN * 128, map, box * 64, kv_row0 + kt * BN, BAR(bfull + s));
+        ++t;
       }
       // no copy may still be landing when the CTA exits
       for (int s = 0; s < NSLOT && s < t; ++s) {
         const int last = s + ((t - 1 - s) / NSLOT) * NSLOT;
-        if (!mbar_test(BAR(C::B_FULL + s), (last / NSLOT) & 1)) {
+        if (!mbar_test(BAR(bfull + s), (last / NSLOT) & 1)) {
           volatile int no_abort = 0;
-          mbar_wait(BAR(C::B_FULL + s), (last / NSLOT) & 1, &no_abort, status, 2, 1ll << 28);
+          mbar_wait(BAR(bfull + s), (last / NSLOT) & 1, &no_abort, status, 2, 1ll << 28);
         }
       }
     }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ UMMA issuer
+  } else if (warp == kSWarp) {
+    // ------------------------------------------------------------ UMMA issuer: S_j = Q K_j^T
     if (lane == 0) {
       StepIter it;
       it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, false);
-      int n = 0, kt;
-      uint32_t bits;
-      while (it.next(kt, bits)) ++n;
       constexpr uint32_t idq = idesc_bf16(BM, BN, 0);
-      constexpr uint32_t idp = idesc_bf16(BM, D, 1);
-      int t = 0;
-      auto wait_full = [&]() -> int {
-        const int s = t % NSLOT, u = t / NSLOT;
-        ++t;
-        return mbar_wait(BAR(C::B_FULL + s), u & 1, abort_flag, status, 3) ? s : -1;
-      };
-      auto issue_s = [&](int j, int s) {
+      bool ok = mbar_wait(BAR(C::B_Q), 0, abort_flag, status, 4);
+      int j = 0, kt;
+      uint32_t bits;
+      while (ok && it.next(kt, bits)) {
+        if (j >= 2) {   // buffer j%2 is free once its softmax group has read S_{j-2}
+          ok = mbar_wait(BAR(C::B_SFREE + (j & 1)), ((j - 2) >> 1) & 1, abort_flag, status, 5);
+          if (!ok) break;
+        }
+        const int s = j % NSLOT;
+        ok = mbar_wait(BAR(C::B_KFULL + s), (j / NSLOT) & 1, abort_flag, status, 3);
+        if (!ok) break;
+        tc_fence_after();
         const uint32_t d = tmem + uint32_t(j & 1) * 128u;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -270,9 +266,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                   smem_desc_sw128(sRing + s * C::T_BYTES + boff, 16, 1024), idq, kk > 0);
         }
         umma_commit(BAR(C::B_S + (j & 1)));
-        umma_commit(BAR(C::B_EMPTY + s));
-      };
-      auto issue_pv = [&](int j, int s) {
+        umma_commit(BAR(C::B_KEMPTY + s));
+        ++j;
+      }
+    }
+  } else if (warp == kPVWarp) {
+    // ------------------------------------------------------------ UMMA issuer: O += P V
+    if (lane == 0) {
+      StepIter it;
+      it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, false);
+      constexpr uint32_t idp = idesc_bf16(BM, D, 1);
+      bool ok = true;
+      int j = 0, kt;
+      uint32_t bits;
+      while (ok && it.next(kt, bits)) {
+        const int s = j % NSLOT;
+        ok = mbar_wait(BAR(C::B_VFULL + s), (j / NSLOT) & 1, abort_flag, status, 3) &&
+             mbar_wait(BAR(C::B_P + (j & 1)), (j >> 1) & 1, abort_flag, status, 6);
+        if (!ok) break;
+        tc_fence_after();
         const uint32_t d = tmem + 256u + uint32_t(j & 1) * D;
         const uint32_t pb = sP + uint32_t(j & 1) * C::P_BYTES;
 #pragma unroll
@@ -280,34 +292,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t aoff = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
           const uint32_t boff = kk * (16 * 128);
           umma_ss(d, smem_desc_sw128(pb + aoff, 16, 1024),
-                  smem_desc_sw128(sRing + s * C::T_BYTES + boff, BN * 128, 1024), idp,
+                  smem_desc_sw128(sVRing + s * C::T_BYTES + boff, BN * 128, 1024), idp,
                   (j >= 2 || kk > 0) ? 1u : 0u);
         }
         umma_commit(BAR(C::B_PV + (j & 1)));
-        umma_commit(BAR(C::B_EMPTY + s));
-      };
-      bool ok = mbar_wait(BAR(C::B_Q), 0, abort_flag, status, 4);
-      for (int j = 0; ok && j < 2 && j < n; ++j) {
-        const int s = wait_full();
-        ok = s >= 0;
-        if (ok) { tc_fence_after(); issue_s(j, s); }
-      }
-      for (int j = 0; ok && j < n; ++j) {
-        if (j + 2 < n) {
-          // S buffer j%2 is free once its softmax group has read S_j
-          ok = mbar_wait(BAR(C::B_SFREE + (j & 1)), (j >> 1) & 1, abort_flag, status, 5);
-          if (!ok) break;
-          const int s = wait_full();
-          ok = s >= 0;
-          if (!ok) break;
-          tc_fence_after();
-          issue_s(j + 2, s);
-        }
-        const int sv = wait_full();
-        ok = sv >= 0 && mbar_wait(BAR(C::B_P + (j & 1)), (j >> 1) & 1, abort_flag, status, 6);
-        if (!ok) break;
-        tc_fence_after();
-        issue_pv(j, sv);
+        umma_commit(BAR(C::B_VEMPTY + s));
+        ++j;
       }
       umma_commit(BAR(C::B_O));
     }
@@ -475,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kSWarp) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
