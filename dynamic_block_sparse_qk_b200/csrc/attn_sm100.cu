@@ -318,11 +318,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     StepIter it;
     it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, false);
     float m_use = -INFINITY, l = 0.f;
-    int j = 0, u = 0, kt;
-    uint32_t bits;
+    int j = grp, u = 0, kt, kt_next;
+    uint32_t bits, bits_next;
     bool ok = true;
-    while (it.next(kt, bits)) {
-      if ((j & 1) != grp) { ++j; continue; }
+    // this group's steps are j = grp, grp + 2, ...: the tile id and mask bits of
+    // the next one are fetched while the current one is processed
+    bool more = it.next(kt_next, bits_next) && (grp == 0 || it.next(kt_next, bits_next));
+    while (more) {
+      kt = kt_next;
+      bits = bits_next;
+      more = it.next(kt_next, bits_next) && it.next(kt_next, bits_next);
       ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_S + grp), u & 1, abort_flag, status, 7));
       if (!ok) break;
       tc_fence_after();
@@ -412,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::B_P + grp));
-      ++j;
+      j += 2;
       ++u;
     }
     // ---- merge the two groups' partial results (every softmax thread gets here once)

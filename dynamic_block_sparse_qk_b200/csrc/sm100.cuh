@@ -25,13 +25,14 @@ __device__ inline void mbar_arrive(uint32_t bar) {
 __device__ inline void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
-// Non-blocking probe of a phase (test_wait never suspends the thread, so a
-// waiter resumes the moment the phase completes).
+// Probe of a phase. try_wait may park the thread in hardware for a short,
+// system-dependent time until the phase completes, which spends less issue
+// bandwidth and power than a tight polling loop.
 __device__ inline bool mbar_test(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred P;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, P;\n\t}"
       : "=r"(ok)
       : "r"(bar), "r"(parity)
