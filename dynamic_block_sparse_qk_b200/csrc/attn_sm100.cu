@@ -13,6 +13,7 @@
 //                      accumulators, as soon as P_j is written. The two issuers
 //                      touch disjoint buffers, so a late V tile never holds up
 //                      the next QK^T and vice versa.
+//   Work order: KV-head major, longest query tiles first within a KV head.
 //   warps 0-3, 4-7     two softmax groups that ping-pong: group g takes the
 //                      steps j with j%2 == g, so one group's exp2 work overlaps
 //                      the other group's TMEM loads, stores and barriers.
@@ -72,6 +73,7 @@ struct StepIter {
   const int32_t* lst[2];
   int cnt[2], pos[2];
   int nsub, kpu, qb0, dense_last, next_kt;
+  int ahead;        // single list: the next entry, already loaded (-2: none)
   int32_t* status;
   bool report;
 
@@ -99,6 +101,8 @@ struct StepIter {
         cnt[i] = c;
       }
     }
+    ahead = -2;
+    if (tile_idx && nsub == 1 && cnt[0] > 0) ahead = lst[0][0];
   }
 
   __device__ bool next(int& kt, uint32_t& bits) {
@@ -110,6 +114,21 @@ struct StepIter {
         for (int ks = 0; ks < kpu; ++ks)
           if (kt * kpu + ks <= qb0 + i) bits |= 1u << (i * kpu + ks);
       return true;
+    }
+    if (nsub == 1) {
+      // one list: the entry was loaded on the previous call, load the next now
+      while (pos[0] < cnt[0]) {
+        const int v = ahead;
+        ++pos[0];
+        ahead = pos[0] < cnt[0] ? lst[0][pos[0]] : -2;
+        if (v >= 0 && v <= qb0) {
+          kt = v / kpu;
+          bits = 1u << (v % kpu);
+          return true;
+        }
+        if (report) report_error(status, CRISP_ERR_DEVICE, v);
+      }
+      return false;
     }
     int best = INT_MAX;
 #pragma unroll
@@ -165,10 +184,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const Workspace W = make_workspace(p);
   int32_t* status = ws_ptr<int32_t>(ws, W.status);
-  const int N = p.seqlen, nb = N / p.block, NT = N / BM, BH = p.batch * p.h_q;
-  const int qt = NT - 1 - int(blockIdx.x) / BH;      // long rows first
-  const int bh = int(blockIdx.x) % BH;
-  const int b = bh / p.h_q, h = bh % p.h_q, hk = h / (p.h_q / p.h_kv);
+  const int N = p.seqlen, nb = N / p.block, NT = N / BM;
+  // Work order: KV-head major (the CTAs running at the same time read the same
+  // K/V stream, which then stays in L2), longest query tiles first inside.
+  const int g = p.h_q / p.h_kv;
+  const int grp_items = g * NT;
+  const int bk = int(blockIdx.x) / grp_items;         // batch * h_kv + kv head
+  const int rem = int(blockIdx.x) % grp_items;
+  const int qt = NT - 1 - rem / g;
+  const int b = bk / p.h_kv, hk = bk % p.h_kv, h = hk * g + rem % g;
+  const int bh = b * p.h_q + h;
   const int row0 = qt * BM;
   const int q_row = bh * N + row0;
   const int kv_row0 = (b * p.h_kv + hk) * N;
@@ -355,7 +380,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mx[e & 3] = fmaxf(mx[e & 3], __uint_as_float(sr[c][e]));
+          for (int e = 0; e < 32; e += 2)
+            mx[(e >> 1) & 3] = max3f(mx[(e >> 1) & 3], __uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]));
       } else {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -383,23 +409,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_PV + grp), (u - 1) & 1, abort_flag, status, 8));
         if (!ok) break;
       }
-      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      // exp2 arguments and row sums two at a time (f32x2), P packed to bf16x2
+      const uint64_t sc2 = pack_f32x2(sl2, sl2), nm2 = pack_f32x2(-mref, -mref);
+      uint64_t acc2[2] = {pack_f32x2(0.f, 0.f), pack_f32x2(0.f, 0.f)};
 #pragma unroll
       for (int ch = 0; ch < 16; ++ch) {          // 16-byte chunk = 8 keys
         uint32_t pk[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float a = fast_exp2(fmaf(__uint_as_float(sr[ch >> 2][(ch & 3) * 8 + 2 * e]), sl2, -mref));
-          const float bq = fast_exp2(fmaf(__uint_as_float(sr[ch >> 2][(ch & 3) * 8 + 2 * e + 1]), sl2, -mref));
-          rs[e] += a + bq;
-          pk[e] = pack_bf16_alu(a, bq);
+          const uint64_t x2 = fma_f32x2(pack_f32x2(__uint_as_float(sr[ch >> 2][(ch & 3) * 8 + 2 * e]),
+                                                   __uint_as_float(sr[ch >> 2][(ch & 3) * 8 + 2 * e + 1])),
+                                        sc2, nm2);
+          float xa, xb;
+          unpack_f32x2(x2, xa, xb);
+          const float a = fast_exp2(xa), bq = fast_exp2(xb);
+          acc2[e & 1] = add_f32x2(acc2[e & 1], pack_f32x2(a, bq));
+          pk[e] = pack_bf16(a, bq);
         }
         const uint32_t addr = prow + uint32_t(ch >> 3) * (BM * 128) + (uint32_t((ch & 7) ^ (r & 7)) << 4);
         asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(pk[0]), "r"(pk[1]),
                      "r"(pk[2]), "r"(pk[3])
                      : "memory");
       }
-      l = l * factor + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+      float r0, r1, r2, r3;
+      unpack_f32x2(acc2[0], r0, r1);
+      unpack_f32x2(acc2[1], r2, r3);
+      l = l * factor + ((r0 + r1) + (r2 + r3));
       if (__any_sync(0xffffffffu, resc)) {
         tc_fence_after();
 #pragma unroll 1
