@@ -321,8 +321,10 @@ def run_sweep(args, out_path):
         torch.cuda.synchronize(dev)
         return e0.elapsed_time(e1) / reps
 
-    for n in SWEEP_N:
-        for f in SWEEP_F:
+    ns = tuple(int(x) for x in args.sweep_n.split(",")) if args.sweep_n else SWEEP_N
+    fs = tuple(float(x) for x in args.sweep_f.split(",")) if args.sweep_f else SWEEP_F
+    for n in ns:
+        for f in fs:
             todo = [a for a in SWEEP_ALPHA if (n, f, a) not in done]
             if not todo:
                 continue
@@ -467,6 +469,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--sweep", default=None, help="write the N x f x alpha sweep to this JSONL file")
+    ap.add_argument("--sweep-n", default=None, help="comma-separated sequence lengths (default: all)")
+    ap.add_argument("--sweep-f", default=None, help="comma-separated diffuse-head fractions (default: all)")
     args = ap.parse_args()
     if args.sweep:
         run_sweep(args, args.sweep)

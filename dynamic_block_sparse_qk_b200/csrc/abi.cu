@@ -23,6 +23,8 @@ int check_params(const crisp_params* p) {
   // the PE softmax partials (ceil(N_b/64) per row) live in a [.][N_b][block] region
   if ((nb + 63) / 64 > p->block) return CRISP_ERR_SHAPE;
   if (static_cast<long long>(p->batch) * p->h_q > 65535) return CRISP_ERR_SHAPE;
+  // TMA tile coordinates are 32-bit: every row of q must be addressable
+  if (static_cast<long long>(p->batch) * p->h_q * p->seqlen >= (1ll << 31)) return CRISP_ERR_SHAPE;
   if (!(p->alpha > 0.f) || !isfinite(p->alpha)) return CRISP_ERR_ARG;
   if (!(p->gamma > 0.f) || p->gamma > 1.f) return CRISP_ERR_ARG;
   if (!isfinite(p->tau_proxy) || !isfinite(p->tau_jsd)) return CRISP_ERR_ARG;

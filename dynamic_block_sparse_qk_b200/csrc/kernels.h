@@ -12,6 +12,9 @@ namespace crisp {
 cudaError_t launch_pool(const crisp_params& p, const void* x, int heads, const int32_t* pattern,
                         int mode, float* out, cudaStream_t st);
 
+// Proxy tile statistics of the last query block (tcgen05 kernel).
+cudaError_t run_proxy_stats(const crisp_params& p, const void* q, const void* k, void* ws, cudaStream_t st);
+
 cudaError_t run_route(const crisp_params& p, const void* q, const void* k, void* ws,
                       int32_t* pattern, float* score, float* p_v, float* p_s, cudaStream_t st);
 

@@ -1,0 +1,358 @@
+// Proxy attention statistics (CRISP paper, Algorithm 2 and Algorithm 3 lines
+// 3-5) on the 5th-generation tensor cores of sm_100a.
+//
+// The proxy rows are the last R = block query rows of a head. For every proxy
+// row r and key tile kb this kernel writes the tile-local row max m (log2
+// units) and the two partial sums of exp2(s - m) over the tile columns c <= r
+// and c > r (the parts of the tile in slash blocks kb and kb + 1), plus, per
+// chunk of kProxyChunk key tiles, the running max / sum a merge pass turns into
+// the proxy normaliser. No b x n proxy map is ever stored.
+//
+// One CTA = one query head and one chunk of key tiles. The UMMA runs with
+// M = 128 on the last 128 query rows (for block 64 the proxy rows are TMEM
+// lanes 64..127) and N = 128 keys per step (one 128-key tile or two 64-key
+// tiles):
+//   warp 8 (one lane)  TMA producer: Q once, then the K tiles (ring).
+//   warp 9 (one lane)  UMMA issuer: S_j = Q K_j^T into TMEM buffer j%2 once
+//                      the softmax group has read S_{j-2}.
+//   warps 0-3, 4-7     two row-statistics groups; group g takes the steps
+//                      j with j%2 == g. Thread r owns TMEM lane r. The row max
+//                      is one pass over the S row, the exp2 sums a second; in
+//                      both the tile split c <= r / c > r is warp-uniform per
+//                      32-column chunk except for the one chunk holding the
+//                      diagonal.
+// Two CTAs fit on an SM (256 TMEM columns and < 100 KB shared memory each).
+// Every mbarrier wait is bounded (status CRISP_ERR_TIMEOUT and a CTA abort
+// flag on expiry); the producer drains its copies before the CTA exits.
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace crisp {
+using namespace sm100;
+
+namespace {
+
+constexpr int PM = 128;                  // UMMA M: query rows held in TMEM
+constexpr int PN = 128;                  // keys per step (UMMA N)
+constexpr int kPxThreads = 320;          // 2 x 4 statistics warps, producer, issuer
+constexpr int kPxProd = 8, kPxMma = 9;
+constexpr uint32_t kPxTmemCols = 256;    // S_0, S_1
+
+template <int D>
+struct PxCfg {
+  static constexpr int NSLOT = D == 128 ? 2 : 4;
+  static constexpr int Q_BYTES = PM * D * 2;
+  static constexpr int T_BYTES = PN * D * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_RING = OFF_Q + Q_BYTES;
+  static constexpr int OFF_XCH = OFF_RING + NSLOT * T_BYTES;    // float[2 groups][2][PM]
+  static constexpr int OFF_BAR = OFF_XCH + 2 * 2 * PM * 4;
+  static constexpr int B_Q = 0, B_KFULL = 1, B_KEMPTY = 1 + NSLOT, B_S = 1 + 2 * NSLOT, B_SFREE = B_S + 2,
+                       N_BARS = B_SFREE + 2;
+  static constexpr int OFF_TMEM = OFF_BAR + 8 * N_BARS;
+  static constexpr int OFF_ABORT = OFF_TMEM + 8;
+  static constexpr int SMEM = OFF_ABORT + 8 + 1024;   // + alignment slack
+  static_assert(2 * (SMEM + 1024) <= 233472, "two CTAs per SM");
+};
+
+template <int D, int R>
+__global__ void __launch_bounds__(kPxThreads, 2)
+    proxy_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                    crisp_params p, void* ws) {
+  using C = PxCfg<D>;
+  constexpr int NSLOT = C::NSLOT;
+  constexpr int KPS = PN / R;          // key tiles per step
+  constexpr int ROW0 = PM - R;         // TMEM lane of proxy row 0
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  unsigned char* gbase = smem_raw + (base - raw);
+  const uint32_t sQ = base + C::OFF_Q, sRing = base + C::OFF_RING;
+  auto BAR = [&](int i) -> uint32_t { return base + C::OFF_BAR + 8u * uint32_t(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::OFF_TMEM);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::OFF_ABORT);
+
+  const Workspace W = make_workspace(p);
+  int32_t* status = ws_ptr<int32_t>(ws, W.status);
+  const int N = p.seqlen, nb = N / R;
+  const int nc = (nb + kProxyChunk - 1) / kProxyChunk;
+  // CTA order: the query heads of one KV head are adjacent, so the CTAs that
+  // run together stream the same K tiles (read from HBM once, then from L2).
+  const int g = p.h_q / p.h_kv;
+  const int hin = int(blockIdx.x) % g;
+  const int t = int(blockIdx.x) / g;
+  const int chunk = t % nc, bk = t / nc;          // bk = batch * h_kv + kv head
+  const int b = bk / p.h_kv, hk = bk % p.h_kv;
+  const int bh = b * p.h_q + hk * g + hin;
+  const int kb0 = chunk * kProxyChunk, kb1 = min(kb0 + kProxyChunk, nb);
+  const int nsteps = (kb1 - kb0 + KPS - 1) / KPS;
+  const int q_row = bh * N + N - PM;
+  const int k_row0 = bk * N + kb0 * R;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(C::B_Q), 1);
+    for (int s = 0; s < NSLOT; ++s) {
+      mbar_init(BAR(C::B_KFULL + s), 1);
+      mbar_init(BAR(C::B_KEMPTY + s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(BAR(C::B_S + i), 1);
+      mbar_init(BAR(C::B_SFREE + i), R / 32);   // one arrival per warp holding proxy rows
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kPxMma) {
+    tmem_alloc(smem_u32(tmem_slot), kPxTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kPxProd && lane == 0) {
+    prefetch_tmap(&tmq);
+    prefetch_tmap(&tmk);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kPxProd) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(BAR(C::B_Q), C::Q_BYTES);
+      for (int box = 0; box < D / 64; ++box) tma_load_2d(sQ + box * PM * 128, &tmq, box * 64, q_row, BAR(C::B_Q));
+      int j = 0;
+      for (; j < nsteps; ++j) {
+        const int s = j % NSLOT, u = j / NSLOT;
+        if (u >= 1 && !mbar_wait(BAR(C::B_KEMPTY + s), (u - 1) & 1, abort_flag, status, 21)) break;
+        mbar_arrive_expect_tx(BAR(C::B_KFULL + s), C::T_BYTES);
+        for (int box = 0; box < D / 64; ++box)
+          tma_load_2d(sRing + s * C::T_BYTES + box * PN * 128, &tmk, box * 64, k_row0 + j * PN,
+                      BAR(C::B_KFULL + s));
+      }
+      // no copy may still be landing when the CTA exits
+      volatile int no_abort = 0;
+      if (!mbar_test(BAR(C::B_Q), 0)) mbar_wait(BAR(C::B_Q), 0, &no_abort, status, 22, 1ll << 28);
+      for (int s = 0; s < NSLOT && s < j; ++s) {
+        const int last = s + ((j - 1 - s) / NSLOT) * NSLOT;
+        if (!mbar_test(BAR(C::B_KFULL + s), (last / NSLOT) & 1))
+          mbar_wait(BAR(C::B_KFULL + s), (last / NSLOT) & 1, &no_abort, status, 22, 1ll << 28);
+      }
+    }
+  } else if (warp == kPxMma) {
+    // ------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idq = idesc_bf16(PM, PN, 0);
+      bool ok = mbar_wait(BAR(C::B_Q), 0, abort_flag, status, 23);
+      for (int j = 0; ok && j < nsteps; ++j) {
+        if (j >= 2) {   // buffer j%2 is free once its group has read S_{j-2}
+          ok = mbar_wait(BAR(C::B_SFREE + (j & 1)), ((j - 2) >> 1) & 1, abort_flag, status, 24);
+          if (!ok) break;
+        }
+        const int s = j % NSLOT;
+        ok = mbar_wait(BAR(C::B_KFULL + s), (j / NSLOT) & 1, abort_flag, status, 25);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t d = tmem + uint32_t(j & 1) * 128u;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * (PM * 128) + (kk & 3) * 32;
+          const uint32_t boff = (kk >> 2) * (PN * 128) + (kk & 3) * 32;
+          umma_ss(d, smem_desc_sw128(sQ + aoff, 16, 1024), smem_desc_sw128(sRing + s * C::T_BYTES + boff, 16, 1024),
+                  idq, kk > 0);
+        }
+        umma_commit(BAR(C::B_S + (j & 1)));
+        umma_commit(BAR(C::B_KEMPTY + s));
+      }
+    }
+  } else if ((warp & 3) * 32 >= ROW0) {
+    // ------------------------------------------------------------ row statistics
+    const int grp = warp >> 2, quad = warp & 3;
+    const int pr = quad * 32 + lane - ROW0;      // proxy row
+    const int mixc = pr >> 5;                    // the 32-column chunk holding column pr (warp-uniform)
+    const int prl = pr & 31;
+    const uint32_t tS = tmem + (uint32_t(quad * 32) << 16) + uint32_t(grp) * 128u;
+    const float sl2 = (p.sm_scale > 0.f ? p.sm_scale : rsqrtf(float(D))) * kLog2e;
+    const uint64_t sc2 = pack_f32x2(sl2, sl2);
+    float* stat_m = ws_ptr<float>(ws, W.stat_m);
+    float* stat_lo = ws_ptr<float>(ws, W.stat_lo);
+    float* stat_hi = ws_ptr<float>(ws, W.stat_hi);
+    float cm = -INFINITY, cl = 0.f;
+
+    // exp2(s * sl2 - mx) summed over one 32-column chunk into lo (columns <= pr)
+    // and hi (columns > pr); `ci` is the chunk index inside its key tile.
+    auto chunk_sums = [&](const uint32_t (&a)[32], int ci, bool last, float mx, uint64_t& lo2, uint64_t& hi2) {
+      const uint64_t nm2 = pack_f32x2(-mx, -mx);
+      if (ci < mixc || (ci > mixc && !last)) {
+        uint64_t acc2[2] = {pack_f32x2(0.f, 0.f), pack_f32x2(0.f, 0.f)};
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const uint64_t x2 = fma_f32x2(pack_f32x2(__uint_as_float(a[e]), __uint_as_float(a[e + 1])), sc2, nm2);
+          float xa, xb;
+          unpack_f32x2(x2, xa, xb);
+          acc2[(e >> 1) & 1] = add_f32x2(acc2[(e >> 1) & 1], pack_f32x2(fast_exp2(xa), fast_exp2(xb)));
+        }
+        const uint64_t sum2 = add_f32x2(acc2[0], acc2[1]);
+        if (ci < mixc) lo2 = add_f32x2(lo2, sum2);
+        else hi2 = add_f32x2(hi2, sum2);
+      } else if (ci == mixc) {
+        float lo = 0.f, hi = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float ex = fast_exp2(fmaf(__uint_as_float(a[e]), sl2, -mx));
+          if (e <= prl) lo += ex;
+          else hi += ex;
+        }
+        lo2 = add_f32x2(lo2, pack_f32x2(lo, 0.f));
+        if (!last) hi2 = add_f32x2(hi2, pack_f32x2(hi, 0.f));
+      }
+    };
+    // max over one chunk (raw scores); on the last key tile only columns <= pr count
+    auto chunk_max = [&](const uint32_t (&a)[32], int ci, bool last, float mx) -> float {
+      if (!last || ci < mixc) {
+        float m2[2] = {mx, -INFINITY};
+#pragma unroll
+        for (int e = 0; e < 32; e += 2)
+          m2[(e >> 1) & 1] = max3f(m2[(e >> 1) & 1], __uint_as_float(a[e]), __uint_as_float(a[e + 1]));
+        return fmaxf(m2[0], m2[1]);
+      }
+      if (ci == mixc) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (e <= prl) mx = fmaxf(mx, __uint_as_float(a[e]));
+      }
+      return mx;
+    };
+    auto finish_tile = [&](int kb, bool last, float mx, uint64_t lo2, uint64_t hi2) {
+      float l0, l1, h0, h1;
+      unpack_f32x2(lo2, l0, l1);
+      unpack_f32x2(hi2, h0, h1);
+      const float lo = l0 + l1, hi = last ? 0.f : h0 + h1;
+      const size_t o = (size_t(bh) * nb + kb) * R + pr;
+      stat_m[o] = mx;
+      stat_lo[o] = lo;
+      stat_hi[o] = hi;
+      const float nm = fmaxf(cm, mx);
+      cl = cl * fast_exp2(cm - nm) + (lo + hi) * fast_exp2(mx - nm);
+      cm = nm;
+    };
+
+    int u = 0;
+    for (int j = grp; j < nsteps; j += 2, ++u) {
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_S + grp), u & 1, abort_flag, status, 26));
+      if (!ok) break;
+      tc_fence_after();
+      const int kbs = kb0 + j * KPS;
+      uint32_t a0[32], a1[32];
+      if constexpr (R == 64) {
+        // two 64-key tiles per step, each one pair of chunks loaded once
+#pragma unroll
+        for (int ks = 0; ks < 2; ++ks) {
+          tmem_ld32(tS + ks * 64, a0);
+          tmem_ld32(tS + ks * 64 + 32, a1);
+          tmem_wait_ld();
+          if (ks == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR(C::B_SFREE + grp));
+          }
+          const int kb = kbs + ks;
+          if (kb < kb1) {
+            const bool last = kb == nb - 1;
+            float mx = chunk_max(a0, 0, last, -INFINITY);
+            mx = chunk_max(a1, 1, last, mx) * sl2;
+            uint64_t lo2 = pack_f32x2(0.f, 0.f), hi2 = pack_f32x2(0.f, 0.f);
+            chunk_sums(a0, 0, last, mx, lo2, hi2);
+            chunk_sums(a1, 1, last, mx, lo2, hi2);
+            finish_tile(kb, last, mx, lo2, hi2);
+          }
+        }
+      } else {
+        // one 128-key tile: a max pass and a sum pass over two pairs of chunks
+        const int kb = kbs;
+        const bool last = kb == nb - 1;
+        tmem_ld32(tS, a0);
+        tmem_ld32(tS + 32, a1);
+        tmem_wait_ld();
+        float mx = chunk_max(a0, 0, last, -INFINITY);
+        mx = chunk_max(a1, 1, last, mx);
+        uint32_t a2[32], a3[32];
+        tmem_ld32(tS + 64, a2);
+        tmem_ld32(tS + 96, a3);
+        tmem_wait_ld();
+        mx = chunk_max(a2, 2, last, mx);
+        mx = chunk_max(a3, 3, last, mx) * sl2;
+        uint64_t lo2 = pack_f32x2(0.f, 0.f), hi2 = pack_f32x2(0.f, 0.f);
+        chunk_sums(a2, 2, last, mx, lo2, hi2);
+        chunk_sums(a3, 3, last, mx, lo2, hi2);
+        tmem_ld32(tS, a0);
+        tmem_ld32(tS + 32, a1);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::B_SFREE + grp));
+        chunk_sums(a0, 0, last, mx, lo2, hi2);
+        chunk_sums(a1, 1, last, mx, lo2, hi2);
+        finish_tile(kb, last, mx, lo2, hi2);
+      }
+    }
+    // ---- merge the two groups' running (max, sum) for this chunk (every
+    // statistics thread gets here exactly once)
+    float* xch = reinterpret_cast<float*>(gbase + C::OFF_XCH);
+    xch[(grp * 2) * PM + pr] = cm;
+    xch[(grp * 2 + 1) * PM + pr] = cl;
+    asm volatile("bar.sync 1, %0;" ::"r"(2 * R) : "memory");
+    if (grp == 0) {
+      const float m1 = xch[2 * PM + pr], l1 = xch[3 * PM + pr];
+      float m = cm, l = cl;
+      if (m1 != -INFINITY) {
+        if (m == -INFINITY) {
+          m = m1;
+          l = l1;
+        } else {
+          const float mm = fmaxf(m, m1);
+          l = l * fast_exp2(m - mm) + l1 * fast_exp2(m1 - mm);
+          m = mm;
+        }
+      }
+      const size_t o = (size_t(bh) * nc + chunk) * R + pr;
+      ws_ptr<float>(ws, W.chunk_m)[o] = m;
+      ws_ptr<float>(ws, W.chunk_l)[o] = l;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kPxMma) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kPxTmemCols);
+  }
+}
+
+template <int D, int R>
+cudaError_t launch_proxy(const crisp_params& p, const void* q, const void* k, void* ws, cudaStream_t st) {
+  CUtensorMap mq, mk;
+  const uint64_t N = uint64_t(p.seqlen);
+  if (!make_tmap(&mq, q, uint64_t(p.batch) * p.h_q * N, D) || !make_tmap(&mk, k, uint64_t(p.batch) * p.h_kv * N, D))
+    return cudaErrorInvalidValue;
+  auto kern = proxy_tc_kernel<D, R>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PxCfg<D>::SMEM);
+  if (e != cudaSuccess) return e;
+  const int nb = p.seqlen / R;
+  const int nc = (nb + kProxyChunk - 1) / kProxyChunk;
+  const unsigned grid = unsigned(p.batch) * p.h_q * nc;
+  kern<<<grid, kPxThreads, PxCfg<D>::SMEM, st>>>(mq, mk, p, ws);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t run_proxy_stats(const crisp_params& p, const void* q, const void* k, void* ws, cudaStream_t st) {
+  if (p.head_dim == 64)
+    return p.block == 64 ? launch_proxy<64, 64>(p, q, k, ws, st) : launch_proxy<64, 128>(p, q, k, ws, st);
+  return p.block == 64 ? launch_proxy<128, 64>(p, q, k, ws, st) : launch_proxy<128, 128>(p, q, k, ws, st);
+}
+
+}  // namespace crisp

@@ -15,145 +15,6 @@
 
 namespace crisp {
 
-// ---------------------------------------------------------------------------
-// Proxy tile statistics. CTA = (chunk of kProxyChunk key tiles, query head).
-// R = block = proxy rows = key-tile width; R/16 warps, 16 proxy rows each.
-// ---------------------------------------------------------------------------
-template <int D, int R>
-__global__ void __launch_bounds__(R * 2) proxy_stats_kernel(const __nv_bfloat16* __restrict__ q,
-                                                            const __nv_bfloat16* __restrict__ k,
-                                                            crisp_params p, void* ws) {
-  constexpr int WARPS = R / 16;
-  constexpr int THREADS = WARPS * 32;
-  constexpr int ROWB = D * 2;          // bytes per row
-  constexpr int CPR = D / 8;           // 16-byte chunks per row
-  constexpr int NT = R / 8;            // n-tiles (8 keys) per key tile
-  extern __shared__ __align__(128) unsigned char smem[];
-  unsigned char* qs = smem;                      // [R][D]
-  unsigned char* ks = smem + R * ROWB;           // [2][R][D]
-
-  const Workspace W = make_workspace(p);
-  const int nb = p.seqlen / p.block;
-  const int nc = (nb + kProxyChunk - 1) / kProxyChunk;
-  const int bh = blockIdx.y;
-  const int b = bh / p.h_q, h = bh % p.h_q;
-  const int hk = h / (p.h_q / p.h_kv);
-  const int chunk = blockIdx.x;
-  const int kb0 = chunk * kProxyChunk;
-  const int kb1 = min(kb0 + kProxyChunk, nb);
-  const size_t N = size_t(p.seqlen);
-  const __nv_bfloat16* qh = q + (size_t(bh) * N + N - R) * D;
-  const __nv_bfloat16* kh = k + (size_t(b) * p.h_kv + hk) * N * D;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const float sl2 = (p.sm_scale > 0.f ? p.sm_scale : rsqrtf(float(D))) * kLog2e;
-
-  auto load_tile = [&](unsigned char* dst, const __nv_bfloat16* src) {
-    const uint32_t base = smem_u32(dst);
-    for (int i = tid; i < R * CPR; i += THREADS) {
-      const int row = i / CPR, c = i % CPR;
-      cp_async16(base + swz(row, c, ROWB), src + size_t(row) * D + c * 8);
-    }
-  };
-  load_tile(qs, qh);
-  load_tile(ks, kh + size_t(kb0) * R * D);
-  cp_async_commit();
-
-  float* stat_m = ws_ptr<float>(ws, W.stat_m);
-  float* stat_lo = ws_ptr<float>(ws, W.stat_lo);
-  float* stat_hi = ws_ptr<float>(ws, W.stat_hi);
-
-  uint32_t qf[D / 16][4];
-  float cm[2] = {-INFINITY, -INFINITY}, cl[2] = {0.f, 0.f};
-  const int g = lane >> 2, t4 = lane & 3;
-
-  for (int kb = kb0; kb < kb1; ++kb) {
-    const int buf = (kb - kb0) & 1;
-    if (kb + 1 < kb1) {
-      load_tile(ks + (buf ^ 1) * R * ROWB, kh + size_t(kb + 1) * R * D);
-    }
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    if (kb == kb0) {
-      const uint32_t qb = smem_u32(qs);
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const int row = warp * 16 + (lane & 15);
-        const int c = kk * 2 + (lane >> 4);
-        ldmatrix_x4(qb + swz(row, c, ROWB), qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3]);
-      }
-    }
-    float acc[NT][4];
-#pragma unroll
-    for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-    const uint32_t kbase = smem_u32(ks + buf * R * ROWB);
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-#pragma unroll
-      for (int j = 0; j < NT; j += 2) {
-        uint32_t b0, b1, b2, b3;
-        const int row = j * 8 + (lane & 7) + ((lane >> 4) << 3);
-        const int c = kk * 2 + ((lane >> 3) & 1);
-        ldmatrix_x4(kbase + swz(row, c, ROWB), b0, b1, b2, b3);
-        mma_bf16_16816(acc[j], qf[kk], b0, b1);
-        mma_bf16_16816(acc[j + 1], qf[kk], b2, b3);
-      }
-    }
-    // Row statistics: rows r0 = warp*16+g and r0+8; tile column c = 8j+2*t4+e.
-    const bool last = (kb == nb - 1);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int r = warp * 16 + g + half * 8;
-      float mx = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < NT; ++j)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = j * 8 + t4 * 2 + e;
-          const float s = acc[j][half * 2 + e] * sl2;
-          if (!last || c <= r) mx = fmaxf(mx, s);
-        }
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-      float lo = 0.f, hi = 0.f;
-#pragma unroll
-      for (int j = 0; j < NT; ++j)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = j * 8 + t4 * 2 + e;
-          const float ex = fast_exp2(acc[j][half * 2 + e] * sl2 - mx);
-          if (c <= r) lo += ex;
-          else if (!last) hi += ex;
-        }
-      lo += __shfl_xor_sync(0xffffffffu, lo, 1);
-      lo += __shfl_xor_sync(0xffffffffu, lo, 2);
-      hi += __shfl_xor_sync(0xffffffffu, hi, 1);
-      hi += __shfl_xor_sync(0xffffffffu, hi, 2);
-      if (t4 == 0) {
-        const size_t o = (size_t(bh) * nb + kb) * R + r;
-        stat_m[o] = mx;
-        stat_lo[o] = lo;
-        stat_hi[o] = hi;
-      }
-      const float nm = fmaxf(cm[half], mx);
-      cl[half] = cl[half] * fast_exp2(cm[half] - nm) + (lo + hi) * fast_exp2(mx - nm);
-      cm[half] = nm;
-    }
-    __syncthreads();
-  }
-  if (t4 == 0) {
-    float* chunk_m = ws_ptr<float>(ws, W.chunk_m);
-    float* chunk_l = ws_ptr<float>(ws, W.chunk_l);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int r = warp * 16 + g + half * 8;
-      const size_t o = (size_t(bh) * nc + chunk) * R + r;
-      chunk_m[o] = cm[half];
-      chunk_l[o] = cl[half];
-    }
-  }
-}
-
 // Row max / normaliser of the proxy map from the chunk partials.
 __global__ void proxy_merge_kernel(crisp_params p, void* ws) {
   const Workspace W = make_workspace(p);
@@ -343,21 +204,6 @@ __global__ void __launch_bounds__(256) route_kernel(const __nv_bfloat16* __restr
 // ---------------------------------------------------------------------------
 // Host launchers.
 // ---------------------------------------------------------------------------
-template <int D, int R>
-static cudaError_t launch_proxy_stats(const crisp_params& p, const void* q, const void* k, void* ws,
-                                      cudaStream_t st) {
-  const int nb = p.seqlen / p.block;
-  const int nc = (nb + kProxyChunk - 1) / kProxyChunk;
-  const size_t smem = size_t(3) * R * D * 2;
-  auto kern = proxy_stats_kernel<D, R>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
-  dim3 grid(nc, p.batch * p.h_q);
-  kern<<<grid, R * 2, smem, st>>>(static_cast<const __nv_bfloat16*>(q),
-                                  static_cast<const __nv_bfloat16*>(k), p, ws);
-  return cudaGetLastError();
-}
-
 cudaError_t launch_pool(const crisp_params& p, const void* x, int heads, const int32_t* pattern,
                         int mode, float* out, cudaStream_t st) {
   const int nb = p.seqlen / p.block;
@@ -374,11 +220,7 @@ cudaError_t run_route(const crisp_params& p, const void* q, const void* k, void*
   const Workspace W = make_workspace(p);
   const int nb = p.seqlen / p.block;
   const int BH = p.batch * p.h_q;
-  cudaError_t e;
-  if (p.head_dim == 64)
-    e = (p.block == 64) ? launch_proxy_stats<64, 64>(p, q, k, ws, st) : launch_proxy_stats<64, 128>(p, q, k, ws, st);
-  else
-    e = (p.block == 64) ? launch_proxy_stats<128, 64>(p, q, k, ws, st) : launch_proxy_stats<128, 128>(p, q, k, ws, st);
+  cudaError_t e = run_proxy_stats(p, q, k, ws, st);
   if (e != cudaSuccess) return e;
   proxy_merge_kernel<<<BH, p.block, 0, st>>>(p, ws);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

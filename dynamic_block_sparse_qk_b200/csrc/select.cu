@@ -225,15 +225,45 @@ __global__ void __launch_bounds__(256) pe_hist_kernel(crisp_params p, const int3
   const int rows_per = 8;
   const int q0 = blockIdx.x * rows_per, q1 = min(q0 + rows_per, nb);
   const uint32_t hi_shift = shift + (level == 2 ? 8 : 12);
+  // The entries of a row are close in value, so the lanes of a warp mostly hit
+  // one or two buckets. Lanes with the same bucket combine first: each lane
+  // links to the next lane of its bucket, five pointer-jumping steps leave the
+  // group's sum in its lowest lane, and only that lane updates shared memory.
+  const int lane = threadIdx.x & 31;
   for (int qb = q0; qb < q1; ++qb) {
     const float* row = abar + size_t(qb) * nb;
-    for (int kb = threadIdx.x; kb <= qb; kb += 256) {
-      const float v = row[kb];
-      const uint32_t u = __float_as_uint(v);
-      if (level > 0 && (u >> hi_shift) != (st.prefix >> hi_shift)) continue;
-      const uint32_t bk = (u >> shift) & uint32_t(nbk - 1);
-      atomicAdd(&hc[bk], 1u);
-      atomicAdd(&hs[bk], double(v));
+    for (int c0 = 0; c0 <= qb; c0 += 256) {          // uniform trip count: the whole CTA iterates
+      const int kb = c0 + int(threadIdx.x);
+      bool take = false;
+      uint32_t bk = 0xFFFFFFFFu;
+      double s = 0.0;
+      if (kb <= qb) {
+        const float v = row[kb];
+        const uint32_t u = __float_as_uint(v);
+        if (level == 0 || (u >> hi_shift) == (st.prefix >> hi_shift)) {
+          take = true;
+          bk = (u >> shift) & uint32_t(nbk - 1);
+          s = double(v);
+        }
+      }
+      if (!__any_sync(0xffffffffu, take)) continue;
+      const unsigned peers = __match_any_sync(0xffffffffu, bk);
+      const unsigned above = lane == 31 ? 0u : peers & (0xFFFFFFFFu << (lane + 1));
+      int nxt = above ? __ffs(above) - 1 : -1;
+#pragma unroll
+      for (int step = 0; step < 5; ++step) {
+        const int src = nxt >= 0 ? nxt : lane;
+        const double o = __shfl_sync(0xffffffffu, s, src);
+        const int on = __shfl_sync(0xffffffffu, nxt, src);
+        if (nxt >= 0) {
+          s += o;
+          nxt = on;
+        }
+      }
+      if (take && (peers & ((1u << lane) - 1u)) == 0u) {
+        atomicAdd(&hc[bk], uint32_t(__popc(peers)));
+        atomicAdd(&hs[bk], s);
+      }
     }
   }
   __syncthreads();

@@ -1,6 +1,7 @@
 // sm_100a primitives written as inline PTX: mbarriers with bounded waits,
 // TMA 2-D tile loads, tcgen05 (TMEM allocation, UMMA issue/commit, TMEM
-// loads/stores, fences) and UMMA shared-memory / instruction descriptors.
+// loads/stores, fences) and UMMA shared-memory / instruction descriptors;
+// on the host, the TMA tensor maps of [rows][d] bf16 matrices.
 #pragma once
 
 #include <cuda.h>
@@ -169,6 +170,37 @@ __host__ __device__ constexpr uint64_t smem_desc_sw128(uint32_t addr, uint32_t l
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(b_mn) << 16) | (uint32_t(N >> 3) << 17) |
          (uint32_t(M >> 4) << 24);
+}
+
+// ----------------------------------------------------------------------------- host: tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// Row-major [rows][d] bf16 matrix, 64-column x 128-row boxes, 128-byte swizzle.
+inline bool make_tmap(CUtensorMap* m, const void* base, uint64_t rows, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(d) * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace sm100

@@ -27,7 +27,10 @@
  *    prefill and clear the word; a caller who runs crisp_select or
  *    crisp_sparse_prefill alone on a new workspace zeroes those 8 bytes.
  *  - Block geometry: N_b = seqlen / block. seqlen must be a multiple of 128
- *    and of block; block is 64 or 128; head_dim is 64 or 128; N_b >= 3.
+ *    and of block; block is 64 or 128; head_dim is 64 or 128;
+ *    3 <= N_b <= 8192 and ceil(N_b / 64) <= block; batch * h_q <= 65535 and
+ *    batch * h_q * seqlen < 2^31 (rows of q addressed by 32-bit tile
+ *    coordinates). Anything else returns CRISP_ERR_SHAPE.
  *  - Return codes: CRISP_OK, or a negative crisp_status. Invalid arguments
  *    never launch a kernel.
  */

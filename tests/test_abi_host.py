@@ -50,6 +50,8 @@ def _p(**kw):
     (dict(alpha=0.0), -1), (dict(gamma=1.5), -1), (dict(gamma=0.0), -1), (dict(k_min_blocks=0), -1),
     (dict(router=7), -1), (dict(vs_rule=2), -1), (dict(sm_scale=-1.0), -1), (dict(batch=0), -2),
     (dict(h_q=32, h_kv=0), -2),
+    # batch * h_q * seqlen = 2^31 query rows: beyond 32-bit tile coordinates
+    (dict(batch=64, h_q=64, h_kv=8, seqlen=2 ** 19), -2),
 ])
 def test_check_params_rejects(lib, kw, code):
     p = _p(**kw)
@@ -59,7 +61,8 @@ def test_check_params_rejects(lib, kw, code):
 
 def test_valid_configs_have_workspace(lib):
     for kw in (dict(), dict(batch=1, h_q=2, h_kv=1, seqlen=2048, head_dim=64, block=64),
-               dict(h_q=28, h_kv=4, seqlen=131072), dict(seqlen=524288)):
+               dict(h_q=28, h_kv=4, seqlen=131072), dict(seqlen=524288),
+               dict(batch=63, h_q=64, h_kv=8, seqlen=2 ** 19)):
         p = _p(**kw)
         assert lib.crisp_check_params(ctypes.byref(p)) == 0
         assert lib.crisp_workspace_size(ctypes.byref(p)) > 0
