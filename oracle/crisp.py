@@ -27,7 +27,7 @@ import numpy as np
 __all__ = [
     "VS", "PE", "CrispParams", "bf16_to_f64", "proxy_attention", "vertical_slash_scores",
     "c_struct_from_map", "route_cstruct", "pooled_estimate_last_block", "js_distance",
-    "route_jsd", "noise_floor", "vs_index_alpha", "vs_index_gamma", "pe_pool",
+    "route_jsd", "noise_floor", "noise_floor_median", "vs_index_alpha", "vs_index_gamma", "pe_pool",
     "pe_estimate", "pe_index", "vs_tile_mask", "vs_tile_mask_tokenwise", "pe_tile_mask",
     "masked_attention_rows", "head_route_and_select", "crisp_prefill",
 ]
@@ -46,7 +46,8 @@ class CrispParams:
     tau_jsd: float = 0.1
     k_min_blocks: int = 8
     router: str = "cstruct"   # "cstruct" (Eq. 2) or "jsd" (Appendix A, Algorithm 5)
-    vs_rule: str = "alpha"    # "alpha" (Algorithm 3) or "gamma" (Appendix A, Algorithm 6)
+    vs_rule: str = "alpha"    # "alpha" (Algorithm 3), "alpha_median" (Algorithm 3 with the
+                              # median floor of Appendix H) or "gamma" (Appendix A, Algorithm 6)
     sm_scale: float = 0.0     # 0 -> 1/sqrt(d)
 
     def scale(self, d: int) -> float:
@@ -167,21 +168,41 @@ def noise_floor(p: np.ndarray) -> np.float32:
     return np.float32(r / np.float32(nb - 2))
 
 
+def noise_floor_median(p: np.ndarray) -> np.float32:
+    """Appendix H, "Median instead of mean as the noise floor" (Table 9): the
+    floor is the median of the non-retained blocks 1..N_b-2 instead of their
+    mean, so one dominant block cannot lift it above weaker genuine signal.
+
+    Reading (the page names the statistic only): the textbook median of the
+    N_b - 2 float32 scores, i.e. the middle value of the sorted scores, or
+    for an even count the mean of the two middle values, (a + b) * 0.5 taken
+    in float32.
+    """
+    mid = np.sort(p.astype(np.float32)[1:-1])
+    m = mid.shape[0]
+    if m % 2:
+        return np.float32(mid[m // 2])
+    return np.float32(np.float32(mid[m // 2 - 1] + mid[m // 2]) * np.float32(0.5))
+
+
 def _topk_desc(values32: np.ndarray, k: int) -> np.ndarray:
     """Indices of the k largest values; equal values -> lower index first."""
     order = np.lexsort((np.arange(values32.shape[0]), -values32.astype(np.float64)))
     return np.sort(order[:k])
 
 
-def vs_index_alpha(p: np.ndarray, alpha: float, k_min: int) -> np.ndarray:
+def vs_index_alpha(p: np.ndarray, alpha: float, k_min: int, floor: str = "mean") -> np.ndarray:
     """Algorithm 3, lines 7-12 for one direction.
 
     k_d = #{j : p[j] > alpha * mu} over all blocks (Eq. 4, strict),
     clipped to [k_min, N_b]; S_d = top-k_d(p). Returns sorted block ids.
+    mu is the mean floor of Eq. 3, or with floor="median" the median floor
+    of Appendix H (Table 9).
     """
     p32 = p.astype(np.float32)
     nb = p32.shape[0]
-    thr = np.float32(np.float32(alpha) * noise_floor(p))
+    mu = noise_floor_median(p) if floor == "median" else noise_floor(p)
+    thr = np.float32(np.float32(alpha) * mu)
     k = int(np.count_nonzero(p32 > thr))
     k = min(max(k, k_min), nb)
     return _topk_desc(p32, k)
@@ -372,9 +393,12 @@ def head_route_and_select(q_head: np.ndarray, k_head: np.ndarray, prm: CrispPara
         if prm.vs_rule == "gamma":
             s_v = vs_index_gamma(p_v, prm.gamma, prm.k_min_blocks)
             s_s = vs_index_gamma(p_s, prm.gamma, prm.k_min_blocks)
+        elif prm.vs_rule in ("alpha", "alpha_median"):
+            floor = "median" if prm.vs_rule == "alpha_median" else "mean"
+            s_v = vs_index_alpha(p_v, prm.alpha, prm.k_min_blocks, floor)
+            s_s = vs_index_alpha(p_s, prm.alpha, prm.k_min_blocks, floor)
         else:
-            s_v = vs_index_alpha(p_v, prm.alpha, prm.k_min_blocks)
-            s_s = vs_index_alpha(p_s, prm.alpha, prm.k_min_blocks)
+            raise ValueError(f"unknown vs_rule {prm.vs_rule!r}")
         out["s_v"], out["s_s"] = s_v, s_s
         out["mask"] = vs_tile_mask(s_v, s_s, nb)
     else:

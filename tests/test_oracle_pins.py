@@ -211,6 +211,75 @@ def test_alpha_rule_hand_cases():
     assert abs(float(O.noise_floor(p)) - 0.0425) < 1e-8
 
 
+def _golden_vectors(name):
+    """Splits a fixture into named vectors: {name: {key: [values, ...]}}."""
+    out, cur = {}, None
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, *vals = line.split()
+            if key == "vector":
+                cur = out.setdefault(vals[0], {})
+            else:
+                cur.setdefault(key, []).append(vals)
+    return out
+
+
+def test_median_floor_hand_cases():
+    vecs = _golden_vectors("median_floor_hand.txt")
+    assert sorted(vecs) == ["A", "B", "C"]
+    for name, g in vecs.items():
+        p = np.array([float(x) for x in g["p"][0]])
+        fl = dict(kv.split("=") for kv in g["floor"][0])
+        assert float(O.noise_floor_median(p)) == float(fl["median"]), name
+        assert abs(float(O.noise_floor(p)) - float(fl["mean"])) < 1e-8, name
+        for vals in g["case"]:
+            kw = dict(kv.split("=") for kv in vals[:3])
+            want = [int(x) for x in vals[4:]]
+            got = O.vs_index_alpha(p, float(kw["alpha"]), int(kw["k_min"]), kw["rule"])
+            assert got.tolist() == want, (name, kw, got)
+
+
+def test_median_floor_is_numpy_median_of_middle_blocks():
+    rng = np.random.default_rng(7)
+    for nb in (3, 4, 5, 64, 257, 4096):
+        p = rng.dirichlet(np.full(nb, 0.3))
+        mid32 = p.astype(np.float32)[1:-1]
+        ref = float(np.median(mid32.astype(np.float64)))
+        got = float(O.noise_floor_median(p))
+        assert abs(got - ref) <= 2 ** -23 * abs(ref) + 1e-45, (nb, got, ref)
+
+
+def test_median_floor_ignores_anchors_and_outlier_size():
+    rng = np.random.default_rng(3)
+    p = rng.dirichlet(np.ones(33))
+    base = float(O.noise_floor_median(p))
+    q = p.copy()
+    q[0], q[-1] = 50.0, 70.0                 # the retained blocks do not enter the floor
+    assert float(O.noise_floor_median(q)) == base
+    # move mass from the sink block into the largest middle block (the scores
+    # still sum to one): the median stays, the mean floor of Eq. 3 rises
+    q = p.copy()
+    j = 1 + int(np.argmax(p[1:-1]))
+    d = 0.5 * p[0]
+    q[j] += d
+    q[0] -= d
+    assert float(O.noise_floor_median(q)) == base
+    assert float(O.noise_floor(q)) > float(O.noise_floor(p)) + 0.4 * d / 31
+
+
+def test_median_floor_equals_mean_floor_on_flat_background():
+    nb = 18
+    p = np.full(nb, 0.5 / (nb - 2))
+    p[0], p[-1] = 0.3, 0.2
+    assert float(O.noise_floor_median(p)) == float(np.float32(0.5 / 16))
+    for a in (0.5, 1.0, 2.0):
+        assert (O.vs_index_alpha(p, a, 2, "median").tolist()
+                == O.vs_index_alpha(p, a, 2, "mean").tolist())
+
+
 def test_noise_floor_clamps_at_zero():
     p = np.array([0.7, 0.0, 0.0, 0.4])   # first + last > 1
     assert float(O.noise_floor(p)) == 0.0
