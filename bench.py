@@ -303,7 +303,7 @@ def run_sweep(args, out_path):
             for line in f:
                 try:
                     d = json.loads(line)
-                    done.add((d["seq_len"], d["diffuse_frac"], d["alpha"]))
+                    done.add((d["seq_len"], d["diffuse_frac"], d["alpha"], d.get("vs_rule", "alpha")))
                 except (ValueError, KeyError):
                     pass
     dev = torch.device("cuda", 0)
@@ -323,9 +323,10 @@ def run_sweep(args, out_path):
 
     ns = tuple(int(x) for x in args.sweep_n.split(",")) if args.sweep_n else SWEEP_N
     fs = tuple(float(x) for x in args.sweep_f.split(",")) if args.sweep_f else SWEEP_F
+    alphas = tuple(float(x) for x in args.sweep_alpha.split(",")) if args.sweep_alpha else SWEEP_ALPHA
     for n in ns:
         for f in fs:
-            todo = [a for a in SWEEP_ALPHA if (n, f, a) not in done]
+            todo = [a for a in alphas if (n, f, a, args.vs_rule) not in done]
             if not todo:
                 continue
             w = sweep_workload(n, f).with_(seed=args.seed)
@@ -336,7 +337,7 @@ def run_sweep(args, out_path):
             pj = C.params_for(q, k, block=w.block, router="jsd")
             pat_j = C.crisp_route(pj, q, k, ws)[0].clone()
             for a in todo:
-                p = C.params_for(q, k, block=w.block, alpha=a)
+                p = C.params_for(q, k, block=w.block, alpha=a, vs_rule=args.vs_rule)
                 out = {}
 
                 def route():
@@ -357,7 +358,7 @@ def run_sweep(args, out_path):
                 nb = w.n_blocks
                 causal = p.batch * p.h_q * nb * (nb + 1) // 2
                 total = t_route + t_select + t_attend
-                rec = {"seq_len": n, "diffuse_frac": f, "alpha": a, "workload": w.name,
+                rec = {"seq_len": n, "diffuse_frac": f, "alpha": a, "vs_rule": args.vs_rule, "workload": w.name,
                        "route_ms": round(t_route, 4), "select_ms": round(t_select, 4),
                        "attend_ms": round(t_attend, 4), "total_ms": round(total, 4),
                        "dense_ms": round(dense_ms, 4), "speedup_vs_dense": round(dense_ms / total, 3),
@@ -463,7 +464,7 @@ def main():
     ap.add_argument("--alpha", type=float, default=1.0)
     ap.add_argument("--gamma", type=float, default=0.95)
     ap.add_argument("--router", default="cstruct")
-    ap.add_argument("--vs-rule", default="alpha")
+    ap.add_argument("--vs-rule", default="alpha", choices=["alpha", "alpha_median", "gamma"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -471,6 +472,7 @@ def main():
     ap.add_argument("--sweep", default=None, help="write the N x f x alpha sweep to this JSONL file")
     ap.add_argument("--sweep-n", default=None, help="comma-separated sequence lengths (default: all)")
     ap.add_argument("--sweep-f", default=None, help="comma-separated diffuse-head fractions (default: all)")
+    ap.add_argument("--sweep-alpha", default=None, help="comma-separated alpha values (default: 0.5,1,2)")
     args = ap.parse_args()
     if args.sweep:
         run_sweep(args, args.sweep)

@@ -20,7 +20,7 @@ CRISP_OK = 0
 STATUS_NAMES = {0: "ok", -1: "invalid argument", -2: "unsupported shape", -3: "workspace too small",
                 -4: "CUDA error", -5: "device wait timed out", -6: "device index out of range"}
 ROUTER = {"cstruct": 0, "jsd": 1}
-VS_RULE = {"alpha": 0, "gamma": 1}
+VS_RULE = {"alpha": 0, "gamma": 1, "alpha_median": 2}
 PATTERN_VS, PATTERN_PE = 0, 1
 
 EXPORTED = ("crisp_version", "crisp_status_string", "crisp_check_params", "crisp_workspace_size",

@@ -30,7 +30,8 @@ int check_params(const crisp_params* p) {
   if (!isfinite(p->tau_proxy) || !isfinite(p->tau_jsd)) return CRISP_ERR_ARG;
   if (p->k_min_blocks < 1) return CRISP_ERR_ARG;
   if (p->router != CRISP_ROUTER_CSTRUCT && p->router != CRISP_ROUTER_JSD) return CRISP_ERR_ARG;
-  if (p->vs_rule != CRISP_VS_ALPHA && p->vs_rule != CRISP_VS_GAMMA) return CRISP_ERR_ARG;
+  if (p->vs_rule != CRISP_VS_ALPHA && p->vs_rule != CRISP_VS_GAMMA && p->vs_rule != CRISP_VS_ALPHA_MEDIAN)
+    return CRISP_ERR_ARG;
   if (!(p->sm_scale >= 0.f) || !isfinite(p->sm_scale)) return CRISP_ERR_ARG;
   return CRISP_OK;
 }

@@ -10,7 +10,8 @@ namespace crisp {
 // ---------------------------------------------------------------------------
 // VS selection, one CTA (1024 threads) per (query head, direction).
 // Scores stay in shared memory. ALPHA: Eq. 4 count, clip, top-k (rank based
-// only when the count is below k_min). GAMMA: rank every block, scatter to
+// only when the count is below k_min); ALPHA_MEDIAN: the same with the median
+// floor of Appendix H (rank selection). GAMMA: rank every block, scatter to
 // descending order, fp64 prefix sum, first prefix >= gamma, clip.
 // Ranks order by value descending, equal values by lower index.
 // ---------------------------------------------------------------------------
@@ -23,6 +24,7 @@ __global__ void __launch_bounds__(1024) vs_select_kernel(crisp_params p, const i
   float* sorted = pv + nb;                                   // [nb] (GAMMA)
   double* scan = reinterpret_cast<double*>(sorted + nb);  // [1024], 8-byte aligned (2*nb floats)
   __shared__ int cnt_s, kcut_s;
+  __shared__ float med_s[2];
   const Workspace W = make_workspace(p);
   const int bh = blockIdx.x, dir = blockIdx.y;
   const float* src = (dir == 0 ? p_v : p_s) + size_t(bh) * nb;
@@ -45,10 +47,30 @@ __global__ void __launch_bounds__(1024) vs_select_kernel(crisp_params p, const i
     return rk;
   };
   int k;
-  if (p.vs_rule == CRISP_VS_ALPHA) {
-    float r = (1.0f - pv[0]) - pv[nb - 1];
-    r = fmaxf(r, 0.0f);
-    const float mu = r / float(nb - 2);
+  if (p.vs_rule == CRISP_VS_ALPHA || p.vs_rule == CRISP_VS_ALPHA_MEDIAN) {
+    float mu;
+    if (p.vs_rule == CRISP_VS_ALPHA) {
+      float r = (1.0f - pv[0]) - pv[nb - 1];
+      r = fmaxf(r, 0.0f);
+      mu = r / float(nb - 2);
+    } else {
+      // Median of the non-retained blocks 1..N_b-2 (Appendix H): the blocks
+      // of ascending rank (m-1)/2 and m/2 among the m = N_b-2 middle scores,
+      // ranks made distinct by the block index.
+      const int m = nb - 2, klo = (m - 1) / 2, khi = m / 2;
+      for (int j = 1 + tid; j < nb - 1; j += 1024) {
+        const float x = pv[j];
+        int rk = 0;
+        for (int i = 1; i < nb - 1; ++i) {
+          const float y = pv[i];
+          rk += (y < x) || (y == x && i < j);
+        }
+        if (rk == klo) med_s[0] = x;
+        if (rk == khi) med_s[1] = x;
+      }
+      __syncthreads();
+      mu = (m & 1) ? med_s[0] : (med_s[0] + med_s[1]) * 0.5f;
+    }
     const float thr = p.alpha * mu;
     int c = 0;
     for (int j = tid; j < nb; j += 1024) c += pv[j] > thr;

@@ -55,7 +55,10 @@ typedef enum {
 } crisp_status;
 
 typedef enum { CRISP_ROUTER_CSTRUCT = 0, CRISP_ROUTER_JSD = 1 } crisp_router;
-typedef enum { CRISP_VS_ALPHA = 0, CRISP_VS_GAMMA = 1 } crisp_vs_rule;
+/* VS selection rule: ALPHA = Algorithm 3 with the mean floor of Eq. 3;
+ * GAMMA = Algorithm 6 (Appendix A); ALPHA_MEDIAN = Algorithm 3 with the
+ * median floor of Appendix H (Table 9). */
+typedef enum { CRISP_VS_ALPHA = 0, CRISP_VS_GAMMA = 1, CRISP_VS_ALPHA_MEDIAN = 2 } crisp_vs_rule;
 typedef enum { CRISP_PATTERN_VS = 0, CRISP_PATTERN_PE = 1 } crisp_pattern;
 
 /* Problem and hyper-parameters (CRISP paper, Section 5 Setup: tau_proxy 0.2,
@@ -103,7 +106,9 @@ int crisp_route(const crisp_params* p, const void* q, const void* k, void* ws, s
 /* Stage (c): index selection and tile lists.
  * VS heads: per direction, Algorithm 3 (vs_rule ALPHA: blocks with
  * p > alpha*mu, mu = max(1-p[0]-p[N_b-1],0)/(N_b-2), count clipped to
- * [k_min, N_b], top-k by score, ties to the lower block) or Algorithm 6
+ * [k_min, N_b], top-k by score, ties to the lower block; vs_rule
+ * ALPHA_MEDIAN: the same with mu = the median of p[1..N_b-2], the mean of
+ * the two middle values for an even count) or Algorithm 6
  * (vs_rule GAMMA: smallest prefix of the descending scores reaching gamma,
  * clipped the same way); the union with vertical block 0 and slash block
  * N_b-1 marks tile (qb, kb <= qb) iff kb is a selected vertical block or

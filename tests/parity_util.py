@@ -58,8 +58,9 @@ def vs_exempt(p: np.ndarray, rule: str, alpha: float, gamma: float, k_min: int) 
     nb = p32.shape[0]
     order = np.lexsort((np.arange(nb), -p32.astype(np.float64)))
     ex = np.zeros(nb, dtype=bool)
-    if rule == "alpha":
-        thr = np.float32(np.float32(alpha) * O.noise_floor(p))
+    if rule in ("alpha", "alpha_median"):
+        mu = O.noise_floor_median(p) if rule == "alpha_median" else O.noise_floor(p)
+        thr = np.float32(np.float32(alpha) * mu)
         ex |= np.abs(p32 - thr) <= EXEMPT_REL * abs(thr)
         cnt = int(np.count_nonzero(p32 > thr))
         if cnt < k_min + int(ex.sum()) and k_min <= nb:

@@ -48,7 +48,7 @@ def _p(**kw):
     (dict(h_q=30), -2), (dict(head_dim=96), -2), (dict(block=32), -2), (dict(seqlen=1000), -2),
     (dict(seqlen=256), -2), (dict(seqlen=2 ** 21), -2), (dict(block=64, seqlen=2 ** 19), -2),
     (dict(alpha=0.0), -1), (dict(gamma=1.5), -1), (dict(gamma=0.0), -1), (dict(k_min_blocks=0), -1),
-    (dict(router=7), -1), (dict(vs_rule=2), -1), (dict(sm_scale=-1.0), -1), (dict(batch=0), -2),
+    (dict(router=7), -1), (dict(vs_rule=3), -1), (dict(sm_scale=-1.0), -1), (dict(batch=0), -2),
     (dict(h_q=32, h_kv=0), -2),
     # batch * h_q * seqlen = 2^31 query rows: beyond 32-bit tile coordinates
     (dict(batch=64, h_q=64, h_kv=8, seqlen=2 ** 19), -2),

@@ -47,6 +47,22 @@ def test_tiny_gamma_vs_rule():          # Abl.1: C_struct routing + gamma VS sel
     _check(WORKLOADS["tiny"], vs_rule="gamma")
 
 
+@pytest.mark.parametrize("alpha", [0.5, 1.0, 2.0])
+def test_tiny_median_floor(alpha):      # Appendix H: median noise floor in the alpha rule
+    _check(WORKLOADS["tiny"], vs_rule="alpha_median", alpha=alpha, expect_both=True)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(seqlen=384, block=128, head_dim=128, h_q=2, h_kv=1),              # N_b = 3: one middle block
+    dict(seqlen=768, block=128, head_dim=64, h_q=4, h_kv=2),               # N_b = 6: even middle count
+    dict(seqlen=1024, block=64, head_dim=128, h_q=3, h_kv=3),              # N_b = 16, B = 64
+])
+def test_edge_shapes_median_floor(kw):
+    base = dict(name="edge", batch=1, n_vertical=2, diffuse_frac=0.5, sink_logit=8.0)
+    base.update(kw)
+    _check(Workload(**base), vs_rule="alpha_median")
+
+
 def test_tiny_jsd_router():             # Abl.2: JSD routing + alpha VS selection
     _check(WORKLOADS["tiny"], router="jsd")
 
@@ -137,6 +153,12 @@ def test_llama_32k():
     vs = [r for r in reps if r["pattern"] == O.VS]
     assert len(vs) == 24
     assert max(r["density"] for r in vs) < 0.2
+
+
+def test_llama_32k_median_floor():
+    w = WORKLOADS["llama_32k"]
+    reps = _check(w, vs_rule="alpha_median", qblocks_fn=lambda b, h: PU.sample_qblocks(w.n_blocks, 2, 1500 + h))
+    assert sum(r["pattern"] == O.VS for r in reps) == 24
 
 
 @pytest.mark.slow
