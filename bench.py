@@ -117,9 +117,10 @@ def max_over_ranks(values, device):
 
 def launches_per_step(router: str) -> dict:
     """Kernels of this library launched by one call of each stage."""
-    route = 4 + (1 if router == "jsd" else 0)      # proxy stats, merge, scores, (K pool), route
-    select = 13                                     # vs select, 2 pools, PE logits/normalise,
-    #                                                 3 x (hist, find), eq count/scan, tiles
+    route = 2 + (2 if router == "jsd" else 0)      # proxy stats (+ merge), scores (+ C_struct route),
+    #                                                 JSD only: K pool, JSD route
+    select = 9                                      # vs select, K/Q pool, PE logits/normalise,
+    #                                                 3 x hist (+ cut), tie count (+ scan), tiles
     return {"route": route, "select": select, "attention": 1, "total": route + select + 1}
 
 

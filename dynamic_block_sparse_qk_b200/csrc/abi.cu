@@ -82,7 +82,8 @@ int crisp_route(const crisp_params* p, const void* q, const void* k, void* ws, s
       !aligned(p_v, 4) || !aligned(p_s, 4))
     return CRISP_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(ws, 0, 8, st);   // a prefill starts: clear the status word
+  // a prefill starts: clear the status word and the per-head completion counters
+  cudaError_t e = cudaMemsetAsync(ws, 0, route_clear_bytes(*p), st);
   if (e == cudaSuccess) e = run_route(*p, q, k, ws, pattern, score, p_v, p_s, st);
   return to_status(e);
 }

@@ -18,11 +18,12 @@ constexpr int kMaxBlocks = 8192;  // N_b limit (selection kernels keep one row i
 // `total` bytes once per problem shape; all stages share it in stream order.
 // ----------------------------------------------------------------------------
 struct Workspace {
-  size_t status;      // int32[64]: [0] status word, [1] first bad index, [8..] counters
+  size_t status;      // int32[64]: [0] status word, [1] first bad index
+  size_t head_cnt;    // uint32[BH][4]: per-head CTA completion counters (proxy, histogram, ties, scores)
   size_t stat_m;      // float[BH][Nb][R]   per-row max of a proxy key tile (log2 units)
   size_t stat_lo;     // float[BH][Nb][R]   sum exp2(s-m) over tile columns c <= r
   size_t stat_hi;     // float[BH][Nb][R]   sum exp2(s-m) over tile columns c >  r
-  size_t chunk_m;     // float[BH][NC][R]   per-row max over a chunk of key tiles
+  size_t chunk_m;     // float[BH][NC][R]   per-row max over a chunk of key tiles (NC = ceil(Nb / proxy_chunk))
   size_t chunk_l;     // float[BH][NC][R]   per-row sum over the chunk (scaled to chunk_m)
   size_t row_m;       // float[BH][R]       proxy row max
   size_t row_l;       // float[BH][R]       proxy row normaliser
@@ -45,7 +46,17 @@ struct PeState {
   double above_sum;    // sum of entries strictly above the decided range
 };
 
-constexpr int kProxyChunk = 32;  // key tiles per proxy CTA
+// Key tiles per proxy CTA: small enough that short sequences still give about
+// four CTAs per SM (148 SMs), at most 32 for long ones; even, so a 128-key
+// step of 64-wide blocks never straddles two chunks.
+__host__ __device__ inline int proxy_chunk(const crisp_params& p) {
+  const long long nb = p.seqlen / p.block;
+  long long c = (nb * p.batch * p.h_q + 591) / 592;
+  c = c < 4 ? 4 : (c > 32 ? 32 : c);
+  return int((c + 1) & ~1ll);
+}
+
+enum HeadCounter { kCntProxy = 0, kCntHist = 1, kCntEq = 2, kCntScores = 3 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -55,11 +66,12 @@ __host__ __device__ inline Workspace make_workspace(const crisp_params& p) {
   const size_t BK = size_t(p.batch) * p.h_kv;
   const size_t nb = size_t(p.seqlen / p.block);
   const size_t R = size_t(p.block);
-  const size_t nc = (nb + kProxyChunk - 1) / kProxyChunk;
+  const size_t nc = (nb + proxy_chunk(p) - 1) / proxy_chunk(p);
   const size_t d = size_t(p.head_dim);
   size_t off = 0;
   auto take = [&](size_t bytes) { size_t o = off; off = align256(off + bytes); return o; };
   w.status = take(64 * 4);
+  w.head_cnt = take(BH * 4 * 4);
   w.stat_m = take(BH * nb * R * 4);
   w.stat_lo = take(BH * nb * R * 4);
   w.stat_hi = take(BH * nb * R * 4);
@@ -77,6 +89,13 @@ __host__ __device__ inline Workspace make_workspace(const crisp_params& p) {
   w.eq_cnt = take(BH * nb * 4);
   w.total = off;
   return w;
+}
+
+// Bytes at the start of the workspace that a routing call clears: the status
+// word and the per-head completion counters (adjacent regions).
+inline size_t route_clear_bytes(const crisp_params& p) {
+  const Workspace w = make_workspace(p);
+  return w.head_cnt + size_t(p.batch) * p.h_q * 4 * 4;
 }
 
 template <typename T>

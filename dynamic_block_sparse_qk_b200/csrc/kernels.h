@@ -9,8 +9,11 @@
 
 namespace crisp {
 
-cudaError_t launch_pool(const crisp_params& p, const void* x, int heads, const int32_t* pattern,
-                        int mode, float* out, cudaStream_t st);
+// Block means of nk K heads into kbar and nq Q heads into qbar, one launch
+// (with a pattern: K heads only where a query head of the group is PE, Q
+// heads only where the head is PE).
+cudaError_t launch_pool(const crisp_params& p, const void* k, const void* q, int nk, int nq,
+                        const int32_t* pattern, float* kbar, float* qbar, cudaStream_t st);
 
 // Proxy tile statistics of the last query block (tcgen05 kernel).
 cudaError_t run_proxy_stats(const crisp_params& p, const void* q, const void* k, void* ws, cudaStream_t st);

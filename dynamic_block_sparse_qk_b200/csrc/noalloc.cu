@@ -73,9 +73,10 @@ extern "C" int crisp_route_noalloc(const crisp_params* p, const void* q, const v
   const int a = scratch_address(&scratch);
   if (a != CRISP_OK) return a;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // The status word must start at zero; every other scratch byte the routing
-  // kernels read is written earlier in the same call.
-  cudaError_t e = cudaMemsetAsync(scratch, 0, 8, st);
+  // The status word and the per-head completion counters must start at zero;
+  // every other scratch byte the routing kernels read is written earlier in
+  // the same call.
+  cudaError_t e = cudaMemsetAsync(scratch, 0, route_clear_bytes(*p), st);
   if (e == cudaSuccess) e = run_route(*p, q, k, scratch, pattern, score, p_v, p_s, st);
   return e == cudaSuccess ? CRISP_OK : CRISP_ERR_CUDA;
 }

@@ -5,8 +5,9 @@
 // row r and key tile kb this kernel writes the tile-local row max m (log2
 // units) and the two partial sums of exp2(s - m) over the tile columns c <= r
 // and c > r (the parts of the tile in slash blocks kb and kb + 1), plus, per
-// chunk of kProxyChunk key tiles, the running max / sum a merge pass turns into
-// the proxy normaliser. No b x n proxy map is ever stored.
+// chunk of proxy_chunk() key tiles, the running max / sum. The last CTA of a
+// head to finish merges the chunks into each proxy row's max and normaliser.
+// No b x n proxy map is ever stored.
 //
 // One CTA = one query head and one chunk of key tiles. The UMMA runs with
 // M = 128 on the last 128 query rows (for block 64 the proxy rows are TMEM
@@ -56,6 +57,23 @@ struct PxCfg {
   static_assert(2 * (SMEM + 1024) <= 233472, "two CTAs per SM");
 };
 
+// Proxy row max and normaliser of head bh from its nc chunk partials, in
+// chunk order. Out of line so that its addresses are not held in registers
+// through the main loop.
+__device__ __noinline__ void merge_chunks(const crisp_params& p, void* ws, int bh, int nc, int R) {
+  const Workspace W = make_workspace(p);
+  const float* cmv = ws_ptr<float>(ws, W.chunk_m) + size_t(bh) * nc * R;
+  const float* clv = ws_ptr<float>(ws, W.chunk_l) + size_t(bh) * nc * R;
+  for (int r = threadIdx.x; r < R; r += blockDim.x) {
+    float m = -INFINITY;
+    for (int c = 0; c < nc; ++c) m = fmaxf(m, __ldcg(cmv + size_t(c) * R + r));
+    float l = 0.f;
+    for (int c = 0; c < nc; ++c) l += __ldcg(clv + size_t(c) * R + r) * fast_exp2(__ldcg(cmv + size_t(c) * R + r) - m);
+    ws_ptr<float>(ws, W.row_m)[size_t(bh) * R + r] = m;
+    ws_ptr<float>(ws, W.row_l)[size_t(bh) * R + r] = l;
+  }
+}
+
 template <int D, int R>
 __global__ void __launch_bounds__(kPxThreads, 2)
     proxy_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
@@ -76,7 +94,8 @@ __global__ void __launch_bounds__(kPxThreads, 2)
   const Workspace W = make_workspace(p);
   int32_t* status = ws_ptr<int32_t>(ws, W.status);
   const int N = p.seqlen, nb = N / R;
-  const int nc = (nb + kProxyChunk - 1) / kProxyChunk;
+  const int chunk_tiles = proxy_chunk(p);
+  const int nc = (nb + chunk_tiles - 1) / chunk_tiles;
   // CTA order: the query heads of one KV head are adjacent, so the CTAs that
   // run together stream the same K tiles (read from HBM once, then from L2).
   const int g = p.h_q / p.h_kv;
@@ -85,7 +104,7 @@ __global__ void __launch_bounds__(kPxThreads, 2)
   const int chunk = t % nc, bk = t / nc;          // bk = batch * h_kv + kv head
   const int b = bk / p.h_kv, hk = bk % p.h_kv;
   const int bh = b * p.h_q + hk * g + hin;
-  const int kb0 = chunk * kProxyChunk, kb1 = min(kb0 + kProxyChunk, nb);
+  const int kb0 = chunk * chunk_tiles, kb1 = min(kb0 + chunk_tiles, nb);
   const int nsteps = (kb1 - kb0 + KPS - 1) / KPS;
   const int q_row = bh * N + N - PM;
   const int k_row0 = bk * N + kb0 * R;
@@ -322,6 +341,7 @@ __global__ void __launch_bounds__(kPxThreads, 2)
     }
   }
 
+  __threadfence();      // this CTA's statistics are visible device-wide before it is counted
   tc_fence_before();
   __syncthreads();
   if (warp == kPxMma) {
@@ -329,6 +349,18 @@ __global__ void __launch_bounds__(kPxThreads, 2)
     tc_fence_after();
     tmem_dealloc(tmem, kPxTmemCols);
   }
+
+  // ---- the last CTA of this head merges the chunk partials into the proxy
+  // row max and normaliser (fixed chunk order: the result does not depend on
+  // which CTA finishes last)
+  volatile int* last = reinterpret_cast<volatile int*>(gbase + C::OFF_ABORT) + 1;
+  uint32_t* cnt = ws_ptr<uint32_t>(ws, make_workspace(p).head_cnt) + size_t(bh) * 4 + kCntProxy;
+  if (threadIdx.x == 0) *last = atomicAdd(cnt, 1u) == uint32_t(nc - 1);
+  __syncthreads();
+  if (!*last) return;
+  __threadfence();
+  merge_chunks(p, ws, bh, nc, R);
+  if (threadIdx.x == 0) *cnt = 0u;   // ready for the next call
 }
 
 template <int D, int R>
@@ -341,7 +373,7 @@ cudaError_t launch_proxy(const crisp_params& p, const void* q, const void* k, vo
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PxCfg<D>::SMEM);
   if (e != cudaSuccess) return e;
   const int nb = p.seqlen / R;
-  const int nc = (nb + kProxyChunk - 1) / kProxyChunk;
+  const int nc = (nb + proxy_chunk(p) - 1) / proxy_chunk(p);
   const unsigned grid = unsigned(p.batch) * p.h_q * nc;
   kern<<<grid, kPxThreads, PxCfg<D>::SMEM, st>>>(mq, mk, p, ws);
   return cudaGetLastError();

@@ -3,87 +3,94 @@
 // (Algorithm 3 lines 3-5), C_struct (Eq. 2) and the JSD router of the
 // paper's Appendix A (Algorithm 5).
 //
-// The b x n proxy map is never stored. One pass computes, for every proxy
-// row r and key tile kb, the tile-local row max m and the two partial sums of
-// exp2(s - m) over tile columns c <= r and c > r. Those two sums are exactly
-// the parts of the tile that fall into slash blocks kb and kb + 1 (the
-// diagonal of entry (r, j) is indexed by j + b - 1 - r). A merge gives each
-// row's max and normaliser, and a final pass turns the tile statistics into
-// p_v and p_s without touching Q or K again.
+// The b x n proxy map is never stored. One tensor-core pass (proxy_sm100.cu)
+// computes, for every proxy row r and key tile kb, the tile-local row max m
+// and the two partial sums of exp2(s - m) over tile columns c <= r and c > r.
+// Those two sums are exactly the parts of the tile that fall into slash
+// blocks kb and kb + 1 (the diagonal of entry (r, j) is indexed by
+// j + b - 1 - r). Its last CTA per head merges them into each row's max and
+// normaliser; the scores pass here turns the tile statistics into p_v and
+// p_s without touching Q or K again.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace crisp {
 
-// Row max / normaliser of the proxy map from the chunk partials.
-__global__ void proxy_merge_kernel(crisp_params p, void* ws) {
-  const Workspace W = make_workspace(p);
-  const int R = p.block, nb = p.seqlen / p.block;
-  const int nc = (nb + kProxyChunk - 1) / kProxyChunk;
-  const int bh = blockIdx.x, r = threadIdx.x;
-  if (r >= R) return;
-  const float* cmv = ws_ptr<float>(ws, W.chunk_m) + size_t(bh) * nc * R;
-  const float* clv = ws_ptr<float>(ws, W.chunk_l) + size_t(bh) * nc * R;
-  float m = -INFINITY;
-  for (int c = 0; c < nc; ++c) m = fmaxf(m, cmv[size_t(c) * R + r]);
-  float l = 0.f;
-  for (int c = 0; c < nc; ++c) l += clv[size_t(c) * R + r] * fast_exp2(cmv[size_t(c) * R + r] - m);
-  ws_ptr<float>(ws, W.row_m)[size_t(bh) * R + r] = m;
-  ws_ptr<float>(ws, W.row_l)[size_t(bh) * R + r] = l;
-}
-
 // p_v[kb] = (1/R) sum_r w(r,kb) (lo+hi);  p_s[kb] = (1/R) sum_r [w(r,kb) lo(kb) + w(r,kb-1) hi(kb-1)]
-// with w(r,kb) = exp2(m(r,kb) - m_r) / l_r. One warp per key block.
+// with w(r,kb) = exp2(m(r,kb) - m_r) / l_r. One warp per key block. With the
+// C_struct router the last CTA of a head also routes it (Eq. 2:
+// C_struct = p_v[0] + p_v[N_b-1], VS iff >= tau_proxy).
 __global__ void proxy_scores_kernel(crisp_params p, void* ws, float* __restrict__ p_v,
-                                    float* __restrict__ p_s) {
+                                    float* __restrict__ p_s, int32_t* __restrict__ pattern,
+                                    float* __restrict__ score) {
+  __shared__ int last;
   const Workspace W = make_workspace(p);
   const int R = p.block, nb = p.seqlen / p.block;
   const int bh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kb = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (kb >= nb) return;
-  const float* sm = ws_ptr<float>(ws, W.stat_m) + size_t(bh) * nb * R;
-  const float* slo = ws_ptr<float>(ws, W.stat_lo) + size_t(bh) * nb * R;
-  const float* shi = ws_ptr<float>(ws, W.stat_hi) + size_t(bh) * nb * R;
-  const float* rm = ws_ptr<float>(ws, W.row_m) + size_t(bh) * R;
-  const float* rl = ws_ptr<float>(ws, W.row_l) + size_t(bh) * R;
-  float sv = 0.f, ss = 0.f;
-  for (int r = lane; r < R; r += 32) {
-    const float il = 1.f / rl[r];
-    const size_t o = size_t(kb) * R + r;
-    const float w = fast_exp2(sm[o] - rm[r]) * il;
-    sv += w * (slo[o] + shi[o]);
-    ss += w * slo[o];
-    if (kb > 0) {
-      const size_t o1 = o - R;
-      ss += fast_exp2(sm[o1] - rm[r]) * il * shi[o1];
+  if (kb < nb) {
+    const float* sm = ws_ptr<float>(ws, W.stat_m) + size_t(bh) * nb * R;
+    const float* slo = ws_ptr<float>(ws, W.stat_lo) + size_t(bh) * nb * R;
+    const float* shi = ws_ptr<float>(ws, W.stat_hi) + size_t(bh) * nb * R;
+    const float* rm = ws_ptr<float>(ws, W.row_m) + size_t(bh) * R;
+    const float* rl = ws_ptr<float>(ws, W.row_l) + size_t(bh) * R;
+    float sv = 0.f, ss = 0.f;
+    for (int r = lane; r < R; r += 32) {
+      const float il = 1.f / rl[r];
+      const size_t o = size_t(kb) * R + r;
+      const float w = fast_exp2(sm[o] - rm[r]) * il;
+      sv += w * (slo[o] + shi[o]);
+      ss += w * slo[o];
+      if (kb > 0) {
+        const size_t o1 = o - R;
+        ss += fast_exp2(sm[o1] - rm[r]) * il * shi[o1];
+      }
+    }
+    sv = warp_sum(sv);
+    ss = warp_sum(ss);
+    if (lane == 0) {
+      p_v[size_t(bh) * nb + kb] = sv / float(R);
+      p_s[size_t(bh) * nb + kb] = ss / float(R);
     }
   }
-  sv = warp_sum(sv);
-  ss = warp_sum(ss);
-  if (lane == 0) {
-    p_v[size_t(bh) * nb + kb] = sv / float(R);
-    p_s[size_t(bh) * nb + kb] = ss / float(R);
-  }
+  if (p.router == CRISP_ROUTER_JSD) return;     // routed by route_kernel after K pooling
+  __threadfence();
+  __syncthreads();
+  uint32_t* cnt = ws_ptr<uint32_t>(ws, W.head_cnt) + size_t(bh) * 4 + kCntScores;
+  if (threadIdx.x == 0) last = atomicAdd(cnt, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last || threadIdx.x != 0) return;
+  __threadfence();
+  const float c = __ldcg(p_v + size_t(bh) * nb) + __ldcg(p_v + size_t(bh) * nb + nb - 1);
+  score[bh] = c;
+  pattern[bh] = (c >= p.tau_proxy) ? CRISP_PATTERN_VS : CRISP_PATTERN_PE;
+  *cnt = 0u;
 }
 
 // ---------------------------------------------------------------------------
 // Block-mean pooling (Algorithm 4 line 3; Algorithm 5 line 3): one CTA per
 // (head, block); 16-byte loads, rows split across thread groups, smem reduce.
-// mode 0: K heads (skipped unless `need` says a query head of the group is
-// PE, or need == NULL); mode 1: Q heads, only PE heads.
+// One launch covers K and Q: rows y < nk of the grid are K heads (skipped
+// unless a query head of the group is PE, or pattern == NULL), the rest Q
+// heads (only PE heads).
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ x,
-                                                   crisp_params p, const int32_t* pattern,
-                                                   int mode, float* __restrict__ out) {
+__global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ k,
+                                                   const __nv_bfloat16* __restrict__ q,
+                                                   crisp_params p, const int32_t* pattern, int nk,
+                                                   float* __restrict__ kbar, float* __restrict__ qbar) {
   constexpr int CPR = D / 8;
   constexpr int RPP = 256 / CPR;   // rows per pass
   __shared__ float part[RPP][D];
   const int R = p.block, nb = p.seqlen / p.block;
-  const int hh = blockIdx.y, kb = blockIdx.x;
+  const int kb = blockIdx.x;
+  const bool is_k = int(blockIdx.y) < nk;
+  const int hh = is_k ? int(blockIdx.y) : int(blockIdx.y) - nk;
+  const __nv_bfloat16* x = is_k ? k : q;
+  float* out = is_k ? kbar : qbar;
   if (pattern) {
-    if (mode == 1) {
+    if (!is_k) {
       if (pattern[hh] != CRISP_PATTERN_PE) return;
     } else {
       const int g = p.h_q / p.h_kv;
@@ -118,9 +125,9 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
 }
 
 // ---------------------------------------------------------------------------
-// Routing: C_struct (Eq. 2, = p_v[0] + p_v[N_b-1]) or the JSD distance
-// (Algorithm 5) between p_v and the pooled estimate softmax(scale *
-// mean(Q_hat) . K_bar[kb]). One CTA (256 threads) per query head.
+// JSD routing (Appendix A, Algorithm 5): the distance between p_v and the
+// pooled estimate softmax(scale * mean(Q_hat) . K_bar[kb]). One CTA (256
+// threads) per query head. (C_struct routing happens in the scores kernel.)
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) route_kernel(const __nv_bfloat16* __restrict__ q,
@@ -136,14 +143,6 @@ __global__ void __launch_bounds__(256) route_kernel(const __nv_bfloat16* __restr
   const int bh = blockIdx.x;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const float* pv = p_v + size_t(bh) * nb;
-  if (p.router != CRISP_ROUTER_JSD) {
-    if (tid == 0) {
-      const float c = pv[0] + pv[nb - 1];
-      score[bh] = c;
-      pattern[bh] = (c >= p.tau_proxy) ? CRISP_PATTERN_VS : CRISP_PATTERN_PE;
-    }
-    return;
-  }
   const float scale = p.sm_scale > 0.f ? p.sm_scale : rsqrtf(float(D));
   const size_t N = size_t(p.seqlen);
   const __nv_bfloat16* qh = q + (size_t(bh) * N + N - R) * D;
@@ -204,14 +203,17 @@ __global__ void __launch_bounds__(256) route_kernel(const __nv_bfloat16* __restr
 // ---------------------------------------------------------------------------
 // Host launchers.
 // ---------------------------------------------------------------------------
-cudaError_t launch_pool(const crisp_params& p, const void* x, int heads, const int32_t* pattern,
-                        int mode, float* out, cudaStream_t st) {
+cudaError_t launch_pool(const crisp_params& p, const void* k, const void* q, int nk, int nq,
+                        const int32_t* pattern, float* kbar, float* qbar, cudaStream_t st) {
+  if (nk + nq == 0) return cudaSuccess;
   const int nb = p.seqlen / p.block;
-  dim3 grid(nb, heads);
+  dim3 grid(nb, nk + nq);
+  const auto* kk = static_cast<const __nv_bfloat16*>(k);
+  const auto* qq = static_cast<const __nv_bfloat16*>(q);
   if (p.head_dim == 64)
-    pool_kernel<64><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), p, pattern, mode, out);
+    pool_kernel<64><<<grid, 256, 0, st>>>(kk, qq, p, pattern, nk, kbar, qbar);
   else
-    pool_kernel<128><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(x), p, pattern, mode, out);
+    pool_kernel<128><<<grid, 256, 0, st>>>(kk, qq, p, pattern, nk, kbar, qbar);
   return cudaGetLastError();
 }
 
@@ -220,16 +222,15 @@ cudaError_t run_route(const crisp_params& p, const void* q, const void* k, void*
   const Workspace W = make_workspace(p);
   const int nb = p.seqlen / p.block;
   const int BH = p.batch * p.h_q;
+  // proxy statistics (+ row merge in the last CTA of each head), block
+  // scores (+ C_struct route in the last CTA of each head)
   cudaError_t e = run_proxy_stats(p, q, k, ws, st);
   if (e != cudaSuccess) return e;
-  proxy_merge_kernel<<<BH, p.block, 0, st>>>(p, ws);
+  proxy_scores_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, ws, p_v, p_s, pattern, score);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  proxy_scores_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, ws, p_v, p_s);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (p.router == CRISP_ROUTER_JSD) {
-    e = launch_pool(p, k, p.batch * p.h_kv, nullptr, 0, ws_ptr<float>(ws, W.kbar), st);
-    if (e != cudaSuccess) return e;
-  }
+  if (p.router != CRISP_ROUTER_JSD) return cudaSuccess;
+  e = launch_pool(p, k, q, p.batch * p.h_kv, 0, nullptr, ws_ptr<float>(ws, W.kbar), nullptr, st);
+  if (e != cudaSuccess) return e;
   const size_t smem = size_t(nb) * 4;
   if (p.head_dim == 64) {
     cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));

@@ -30,6 +30,20 @@ __global__ void __launch_bounds__(1024) vs_select_kernel(crisp_params p, const i
   const float* src = (dir == 0 ? p_v : p_s) + size_t(bh) * nb;
   uint8_t* sel = ws_ptr<uint8_t>(ws, W.sel) + (size_t(bh) * 2 + dir) * nb;
   const int tid = threadIdx.x;
+  // Fresh state for this head's PE path, which runs after this kernel in
+  // stream order: radix-select histograms (half per direction CTA), the cut
+  // state and the completion counters of the histogram and tie kernels.
+  {
+    uint32_t* hc = ws_ptr<uint32_t>(ws, W.hist_cnt) + size_t(bh) * 4096 + dir * 2048;
+    double* hs = ws_ptr<double>(ws, W.hist_sum) + size_t(bh) * 4096 + dir * 2048;
+    for (int i = tid; i < 2048; i += 1024) { hc[i] = 0u; hs[i] = 0.0; }
+    if (dir == 0 && tid == 0) {
+      ws_ptr<PeState>(ws, W.pe_state)[bh] = PeState{};
+      uint32_t* cnt = ws_ptr<uint32_t>(ws, W.head_cnt) + size_t(bh) * 4;
+      cnt[kCntHist] = 0u;
+      cnt[kCntEq] = 0u;
+    }
+  }
   if (pattern[bh] != CRISP_PATTERN_VS) {
     for (int j = tid; j < nb; j += 1024) sel[j] = 0;
     return;
@@ -229,6 +243,69 @@ __device__ inline void level_geom(int level, int& shift, int& nbk) {
   nbk = level == 2 ? 256 : 4096;
 }
 
+// The highest bucket whose descending cumulative sum (above_sum + buckets
+// above + itself) reaches gamma; run by the 256 threads of the last histogram
+// CTA of a head. suf: 256 doubles of shared scratch, ctl: 2 ints.
+__device__ void pe_find(const crisp_params& p, PeState* stp, uint32_t* gc, double* gs, int level,
+                        double* suf, int* ctl) {
+  int shift, nbk;
+  level_geom(level, shift, nbk);
+  const int tid = threadIdx.x;
+  const int per = nbk / 256;   // 16 (levels 0, 1) or 1 (level 2)
+  int& best = ctl[0];
+  int& lowest = ctl[1];
+  // thread t owns buckets counted from the top: nbk-1 - (t*per + i)
+  double own = 0.0;
+  for (int i = 0; i < per; ++i) own += __ldcg(gs + (nbk - 1 - (tid * per + i)));
+  suf[tid] = own;
+  if (tid == 0) { best = -1; lowest = 1 << 30; }
+  __syncthreads();
+  for (int bk = tid; bk < nbk; bk += 256)
+    if (__ldcg(gc + bk)) atomicMin(&lowest, bk);
+  for (int off = 1; off < 256; off <<= 1) {
+    const double v = tid >= off ? suf[tid - off] : 0.0;
+    __syncthreads();
+    suf[tid] += v;
+    __syncthreads();
+  }
+  const double g = double(p.gamma);
+  const double above0 = stp->above_sum;
+  double run = above0 + (tid > 0 ? suf[tid - 1] : 0.0);
+  for (int i = 0; i < per; ++i) {
+    const int bk = nbk - 1 - (tid * per + i);
+    const double v = __ldcg(gs + bk);
+    if (run + v >= g) { atomicMax(&best, bk); break; }
+    run += v;
+  }
+  __syncthreads();
+  // Recompute the sum strictly above the chosen bucket (single thread, exact order).
+  if (tid == 0) {
+    PeState s = *stp;
+    int cut = best;
+    if (cut < 0 && level > 0 && lowest < nbk) cut = lowest;  // rounding fell short: whole range
+    if (cut < 0) {
+      s.all = 1;                       // the whole triangle sums below gamma
+    } else {
+      double above = above0;
+      for (int bk = nbk - 1; bk > cut; --bk) above += __ldcg(gs + bk);
+      s.prefix |= uint32_t(cut) << shift;
+      s.above_sum = above;
+      if (level == 2) {
+        const float tv = __uint_as_float(s.prefix);
+        const double need = g - above;
+        double m = ceil(need / double(tv));
+        if (m < 1.0) m = 1.0;
+        const double cap = double(__ldcg(gc + cut));
+        if (m > cap) m = cap;
+        s.m_equal = uint32_t(m);
+      }
+    }
+    *stp = s;
+  }
+  __syncthreads();
+  for (int i = tid; i < nbk; i += 256) { gc[i] = 0; gs[i] = 0.0; }
+}
+
 __global__ void __launch_bounds__(256) pe_hist_kernel(crisp_params p, const int32_t* pattern,
                                                       void* ws, int level) {
   __shared__ uint32_t hc[4096];
@@ -293,118 +370,56 @@ __global__ void __launch_bounds__(256) pe_hist_kernel(crisp_params p, const int3
   double* gs = ws_ptr<double>(ws, W.hist_sum) + size_t(bh) * 4096;
   for (int i = threadIdx.x; i < nbk; i += 256)
     if (hc[i]) { atomicAdd(&gc[i], hc[i]); atomicAdd(&gs[i], hs[i]); }
+  // The last CTA of this head to finish finds the cut bucket.
+  __threadfence();
+  __syncthreads();
+  int* ctl = reinterpret_cast<int*>(hc);       // the shared histogram is free now
+  uint32_t* cnt = ws_ptr<uint32_t>(ws, W.head_cnt) + size_t(bh) * 4 + kCntHist;
+  if (threadIdx.x == 0) ctl[0] = atomicAdd(cnt, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!ctl[0]) return;
+  __threadfence();
+  pe_find(p, ws_ptr<PeState>(ws, W.pe_state) + bh, gc, gs, level, hs, ctl + 1);
+  if (threadIdx.x == 0) *cnt = 0u;
 }
 
-// One CTA (1024 threads) per PE head: the highest bucket whose descending
-// cumulative sum (above_sum + buckets above + itself) reaches gamma.
-__global__ void __launch_bounds__(1024) pe_find_kernel(crisp_params p, const int32_t* pattern,
-                                                       void* ws, int level) {
-  __shared__ double suf[1024];
-  __shared__ int best, lowest;
-  const Workspace W = make_workspace(p);
-  const int bh = blockIdx.x;
-  if (pattern[bh] != CRISP_PATTERN_PE) return;
-  PeState* stp = ws_ptr<PeState>(ws, W.pe_state) + bh;
-  if (stp->all) return;
-  int shift, nbk;
-  level_geom(level, shift, nbk);
-  uint32_t* gc = ws_ptr<uint32_t>(ws, W.hist_cnt) + size_t(bh) * 4096;
-  double* gs = ws_ptr<double>(ws, W.hist_sum) + size_t(bh) * 4096;
-  const int tid = threadIdx.x;
-  const int per = nbk / 1024 > 0 ? nbk / 1024 : 1;   // 4 (levels 0,1) or 1 (level 2)
-  // thread t owns buckets [hi .. lo] counted from the top: top index = nbk-1 - t*per
-  double own = 0.0;
-  for (int i = 0; i < per; ++i) {
-    const int bk = nbk - 1 - (tid * per + i);
-    if (bk >= 0) own += gs[bk];
-  }
-  suf[tid] = own;
-  if (tid == 0) { best = -1; lowest = 1 << 30; }
-  __syncthreads();
-  for (int bk = tid; bk < nbk; bk += 1024)
-    if (gc[bk]) atomicMin(&lowest, bk);
-  for (int off = 1; off < 1024; off <<= 1) {
-    const double v = tid >= off ? suf[tid - off] : 0.0;
-    __syncthreads();
-    suf[tid] += v;
-    __syncthreads();
-  }
-  const double g = double(p.gamma);
-  const double above0 = stp->above_sum;
-  double run = above0 + (tid > 0 ? suf[tid - 1] : 0.0);
-  for (int i = 0; i < per; ++i) {
-    const int bk = nbk - 1 - (tid * per + i);
-    if (bk < 0) break;
-    if (run + gs[bk] >= g) { atomicMax(&best, bk); break; }
-    run += gs[bk];
-  }
-  __syncthreads();
-  // Recompute the sum strictly above the chosen bucket (single thread, exact order).
-  if (tid == 0) {
-    PeState s = *stp;
-    int cut = best;
-    if (cut < 0 && level > 0 && lowest < nbk) cut = lowest;  // rounding fell short: whole range
-    if (cut < 0) {
-      s.all = 1;                       // the whole triangle sums below gamma
-    } else {
-      const int best = cut;
-      double above = above0;
-      for (int bk = nbk - 1; bk > best; --bk) above += gs[bk];
-      s.prefix |= uint32_t(best) << shift;
-      s.above_sum = above;
-      if (level == 2) {
-        const float tv = __uint_as_float(s.prefix);
-        const double need = g - above;
-        double m = ceil(need / double(tv));
-        if (m < 1.0) m = 1.0;
-        const double cap = double(gc[best]);
-        if (m > cap) m = cap;
-        s.m_equal = uint32_t(m);
-      }
-    }
-    *stp = s;
-  }
-  __syncthreads();
-  for (int i = tid; i < nbk; i += 1024) { gc[i] = 0; gs[i] = 0.0; }
-}
-
-// Per-row count of entries equal to the cut value, then an exclusive scan
-// per head, so the tile builder can take the first m_equal of them in flat
-// (row-major) order.
-__global__ void pe_eqcount_kernel(crisp_params p, const int32_t* pattern, void* ws) {
+// Per-row count of entries equal to the cut value; the last CTA of a head
+// turns the counts into an exclusive scan, so the tile builder can take the
+// first m_equal of them in flat (row-major) order.
+__global__ void __launch_bounds__(256) pe_eqcount_kernel(crisp_params p, const int32_t* pattern, void* ws) {
+  __shared__ uint32_t part[256];
+  __shared__ int last;
   const Workspace W = make_workspace(p);
   const int nb = p.seqlen / p.block;
   const int bh = blockIdx.y;
   if (pattern[bh] != CRISP_PATTERN_PE) return;
   const PeState st = ws_ptr<PeState>(ws, W.pe_state)[bh];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qb = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (qb >= nb || st.all) return;
-  const float tv = __uint_as_float(st.prefix);
-  const float* row = ws_ptr<float>(ws, W.abar) + (size_t(bh) * nb + qb) * nb;
-  uint32_t c = 0;
-  for (int kb = lane; kb <= qb; kb += 32) c += row[kb] == tv;
-  c = __reduce_add_sync(0xffffffffu, c);
-  if (lane == 0) ws_ptr<uint32_t>(ws, W.eq_cnt)[size_t(bh) * nb + qb] = c;
-}
-
-__global__ void __launch_bounds__(1024) pe_eqscan_kernel(crisp_params p, const int32_t* pattern,
-                                                         void* ws) {
-  __shared__ uint32_t part[1024];
-  const Workspace W = make_workspace(p);
-  const int nb = p.seqlen / p.block;
-  const int bh = blockIdx.x;
-  if (pattern[bh] != CRISP_PATTERN_PE) return;
-  if (ws_ptr<PeState>(ws, W.pe_state)[bh].all) return;
+  if (st.all) return;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qb = blockIdx.x * 8 + warp;
   uint32_t* ec = ws_ptr<uint32_t>(ws, W.eq_cnt) + size_t(bh) * nb;
-  const int tid = threadIdx.x;
-  const int per = (nb + 1023) / 1024;
-  const int j0 = tid * per, j1 = min(j0 + per, nb);
+  if (qb < nb) {
+    const float tv = __uint_as_float(st.prefix);
+    const float* row = ws_ptr<float>(ws, W.abar) + (size_t(bh) * nb + qb) * nb;
+    uint32_t c = 0;
+    for (int kb = lane; kb <= qb; kb += 32) c += row[kb] == tv;
+    c = __reduce_add_sync(0xffffffffu, c);
+    if (lane == 0) ec[qb] = c;
+  }
+  __threadfence();
+  __syncthreads();
+  uint32_t* cnt = ws_ptr<uint32_t>(ws, W.head_cnt) + size_t(bh) * 4 + kCntEq;
+  if (tid == 0) last = atomicAdd(cnt, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  const int per = (nb + 255) / 256;
+  const int j0 = min(tid * per, nb), j1 = min(j0 + per, nb);
   uint32_t s = 0;
-  for (int j = j0; j < j1; ++j) s += ec[j];
+  for (int j = j0; j < j1; ++j) s += __ldcg(ec + j);
   part[tid] = s;
   __syncthreads();
-  for (int off = 1; off < 1024; off <<= 1) {
+  for (int off = 1; off < 256; off <<= 1) {
     const uint32_t v = tid >= off ? part[tid - off] : 0u;
     __syncthreads();
     part[tid] += v;
@@ -412,10 +427,11 @@ __global__ void __launch_bounds__(1024) pe_eqscan_kernel(crisp_params p, const i
   }
   uint32_t run = tid > 0 ? part[tid - 1] : 0u;
   for (int j = j0; j < j1; ++j) {
-    const uint32_t c = ec[j];
+    const uint32_t c = __ldcg(ec + j);
     ec[j] = run;
     run += c;
   }
+  if (tid == 0) *cnt = 0u;
 }
 
 // ---------------------------------------------------------------------------
@@ -539,12 +555,11 @@ cudaError_t run_select(const crisp_params& p, const void* q, const void* k, cons
     vs_select_kernel<<<dim3(BH, 2), 1024, smem, st>>>(p, pattern, p_v, p_s, ws);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  // (2) PE path: pooling, estimate, gamma cut.
-  if (p.router != CRISP_ROUTER_JSD) {
-    e = launch_pool(p, k, p.batch * p.h_kv, pattern, 0, ws_ptr<float>(ws, W.kbar), st);
-    if (e != cudaSuccess) return e;
-  }
-  e = launch_pool(p, q, BH, pattern, 1, ws_ptr<float>(ws, W.qbar), st);
+  // (2) PE path: pooling (K where the router has not pooled it already, Q of
+  // PE heads), estimate, gamma cut (three radix levels, each with its cut
+  // found by the last histogram CTA of the head), ties at the cut value.
+  e = launch_pool(p, k, q, p.router == CRISP_ROUTER_JSD ? 0 : p.batch * p.h_kv, BH, pattern,
+                  ws_ptr<float>(ws, W.kbar), ws_ptr<float>(ws, W.qbar), st);
   if (e != cudaSuccess) return e;
   {
     const int nt = (nb + 63) / 64;
@@ -555,18 +570,11 @@ cudaError_t run_select(const crisp_params& p, const void* q, const void* k, cons
     pe_normalize_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, pattern, ws);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  if ((e = cudaMemsetAsync(ws_ptr<char>(ws, W.hist_cnt), 0, size_t(BH) * 4096 * 4, st)) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(ws_ptr<char>(ws, W.hist_sum), 0, size_t(BH) * 4096 * 8, st)) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(ws_ptr<char>(ws, W.pe_state), 0, size_t(BH) * sizeof(PeState), st)) != cudaSuccess) return e;
   for (int level = 0; level < 3; ++level) {
     pe_hist_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, pattern, ws, level);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    pe_find_kernel<<<BH, 1024, 0, st>>>(p, pattern, ws, level);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   pe_eqcount_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, pattern, ws);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  pe_eqscan_kernel<<<BH, 1024, 0, st>>>(p, pattern, ws);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // (3) tile lists.
   build_tiles_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, pattern, ws, mask, tile_idx, tile_cnt);

@@ -24,8 +24,10 @@
  *    an out-of-range tile index) are recorded in a status word held in the
  *    first 8 bytes of `ws`, read back (and cleared) with
  *    crisp_get_device_status(). crisp_route and crisp_dense_prefill start a
- *    prefill and clear the word; a caller who runs crisp_select or
- *    crisp_sparse_prefill alone on a new workspace zeroes those 8 bytes.
+ *    prefill and clear the word (crisp_route also clears the per-head
+ *    completion counters its kernels keep right after it); a caller who runs
+ *    crisp_select or crisp_sparse_prefill alone on a new workspace zeroes
+ *    those 8 bytes.
  *  - Block geometry: N_b = seqlen / block. seqlen must be a multiple of 128
  *    and of block; block is 64 or 128; head_dim is 64 or 128;
  *    3 <= N_b <= 8192 and ceil(N_b / 64) <= block; batch * h_q <= 65535 and
