@@ -15,6 +15,12 @@ Readings of steps the paper leaves open (each is stated where it is used):
   * decisions (route, threshold compare, top-k, gamma cut) are taken on
     float32 values, the kernel's precision; the scores feeding them are
     computed in float64 and rounded once.
+  * n need not be a multiple of B: Section 4.3 partitions the map into
+    N_b = ceil(n / B) blocks, so the last block holds n - (N_b - 1) B
+    tokens. Q_hat is still the last B query rows (Algorithm 2 takes the last
+    b rows, a count); block sums and block means run over the tokens a block
+    holds; the anchors of Eq. 2 stay the first and last block of the
+    partition, so C_struct = p_v[0] + p_v[N_b - 1] as in Algorithm 3.
 """
 from __future__ import annotations
 
@@ -25,7 +31,7 @@ from typing import Dict, List, Optional, Sequence
 import numpy as np
 
 __all__ = [
-    "VS", "PE", "CrispParams", "bf16_to_f64", "proxy_attention", "vertical_slash_scores",
+    "VS", "PE", "CrispParams", "bf16_to_f64", "n_blocks", "proxy_attention", "vertical_slash_scores",
     "c_struct_from_map", "route_cstruct", "pooled_estimate_last_block", "js_distance",
     "route_jsd", "noise_floor", "noise_floor_median", "vs_index_alpha", "vs_index_gamma", "pe_pool",
     "pe_estimate", "pe_index", "vs_tile_mask", "vs_tile_mask_tokenwise", "pe_tile_mask",
@@ -81,6 +87,20 @@ def proxy_attention(q_hat: np.ndarray, k: np.ndarray, scale: float) -> np.ndarra
     return e / e.sum(axis=1, keepdims=True)
 
 
+def n_blocks(n: int, block: int) -> int:
+    """N_b = ceil(n / B) (Section 4.3)."""
+    return -(-n // block)
+
+
+def _block_sums(x: np.ndarray, block: int) -> np.ndarray:
+    """Sum of x over each block of the N_b = ceil(n / B) partition of axis 0
+    (the last block may hold fewer than B entries)."""
+    n = x.shape[0]
+    nb = n_blocks(n, block)
+    pad = np.zeros((nb * block - n,) + x.shape[1:], dtype=x.dtype)
+    return np.concatenate([x, pad]).reshape((nb, block) + x.shape[1:]).sum(axis=1)
+
+
 def vertical_slash_scores(a_hat: np.ndarray, block: int):
     """Block scores p_v, p_s of Algorithm 3, lines 3-5.
 
@@ -90,14 +110,13 @@ def vertical_slash_scores(a_hat: np.ndarray, block: int):
     blockpool: sum of the per-key (per-diagonal) means inside each block.
     """
     b, n = a_hat.shape
-    nb = n // block
     a_v = a_hat.mean(axis=0)
     a_s = np.zeros(n)
     for r in range(b):
         shift = b - 1 - r
         a_s[shift:] += a_hat[r, : n - shift]
     a_s /= b
-    return a_v.reshape(nb, block).sum(axis=1), a_s.reshape(nb, block).sum(axis=1)
+    return _block_sums(a_v, block), _block_sums(a_s, block)
 
 
 def c_struct_from_map(a_hat: np.ndarray, block: int) -> float:
@@ -105,12 +124,13 @@ def c_struct_from_map(a_hat: np.ndarray, block: int) -> float:
 
     Anchors: the sink window (first block) and the local recency window
     (last block); Section 4.3 states these windows are exactly the first and
-    last block (reading at B=64: one block, not 128 tokens).
+    last block (reading at B=64: one block, not 128 tokens; for a partial
+    last block, that block: keys (N_b - 1) B .. n - 1).
     """
     b, n = a_hat.shape
     anchors = np.zeros(n, dtype=bool)
     anchors[:block] = True
-    anchors[n - block:] = True
+    anchors[(n_blocks(n, block) - 1) * block:] = True
     return float(a_hat[:, anchors].sum() / b)
 
 
@@ -128,8 +148,7 @@ def pooled_estimate_last_block(q_hat: np.ndarray, k: np.ndarray, block: int, sca
     pool = block mean. The last query block sees every key block, so no
     block-level causal mask applies.
     """
-    n, d = k.shape
-    k_bar = k.reshape(n // block, block, d).mean(axis=1)
+    k_bar = pe_pool(k, block)
     q_bar = q_hat.mean(axis=0)
     z = (k_bar @ q_bar) * scale
     z = z - z.max()
@@ -234,9 +253,11 @@ def vs_index_gamma(p: np.ndarray, gamma: float, k_min: int) -> np.ndarray:
 # (c) Pooled estimation for diffuse heads — Algorithm 4 (PE Index).
 # ---------------------------------------------------------------------------
 def pe_pool(x: np.ndarray, block: int) -> np.ndarray:
-    """Algorithm 4, line 3: block-mean pooling over all rows ([n, d] -> [N_b, d])."""
-    n, d = x.shape
-    return x.reshape(n // block, block, d).mean(axis=1)
+    """Algorithm 4, line 3: block-mean pooling over all rows ([n, d] -> [N_b, d]);
+    a partial last block is the mean of the rows it holds."""
+    n = x.shape[0]
+    counts = np.minimum(block, n - block * np.arange(n_blocks(n, block)))
+    return _block_sums(x, block) / counts[:, None]
 
 
 def pe_estimate(q_bar: np.ndarray, k_bar: np.ndarray, scale: float) -> np.ndarray:
@@ -273,7 +294,8 @@ def pe_index(a_bar: np.ndarray, gamma: float) -> np.ndarray:
 # ---------------------------------------------------------------------------
 # (d) Tile masks and masked attention — Eq. 1.
 # ---------------------------------------------------------------------------
-def vs_tile_mask(s_v: Sequence[int], s_s: Sequence[int], nb: int) -> np.ndarray:
+def vs_tile_mask(s_v: Sequence[int], s_s: Sequence[int], nb: int, n: Optional[int] = None,
+                 block: Optional[int] = None) -> np.ndarray:
     """Tile (qb, kb) of a VS head is computed iff it holds a selected entry.
 
     Algorithm 3 returns S_v U S_s U {0, N_b-1}: vertical block ids and slash
@@ -282,7 +304,12 @@ def vs_tile_mask(s_v: Sequence[int], s_s: Sequence[int], nb: int) -> np.ndarray:
     Slash block jb covers key-query offsets [ob*B, ob*B + B - 1] with
     ob = N_b - 1 - jb, which meet tile (qb, kb) exactly when qb - kb is ob or
     ob + 1. Tiles are computed whole (plus the causal mask in-tile).
+
+    With n given and not a multiple of B the offsets of a slash block are no
+    longer aligned to tiles (see _vs_tile_mask_ragged).
     """
+    if n is not None and n != nb * block:
+        return _vs_tile_mask_ragged(s_v, s_s, n, block)
     col = np.zeros(nb, dtype=bool)
     col[np.asarray(s_v, dtype=np.int64)] = True
     col[0] = True
@@ -298,6 +325,39 @@ def vs_tile_mask(s_v: Sequence[int], s_s: Sequence[int], nb: int) -> np.ndarray:
     return causal & (col[None, :] | off[d0] | off[d1])
 
 
+def _vs_tile_mask_ragged(s_v, s_s, n: int, block: int) -> np.ndarray:
+    """The VS tile rule for a sequence whose last block is partial.
+
+    Pair (t, j), j <= t, lies on slash index j + n - 1 - t. With
+    s = (n - 1) mod B, t = qb B + r and j = kb B + c this is
+    (N_b - 1 - delta) B + s + (c - r), delta = qb - kb. Over the pairs of a
+    tile, c - r takes every value in [-(R_q - 1), C_k - 1] (R_q, C_k: rows /
+    keys of the two blocks) off the diagonal and [-(R_q - 1), 0] on it, so
+    the tile meets the consecutive slash blocks
+    N_b - 1 - delta + floor((s + v) / B) for v between those bounds: up to
+    three of them, where aligned blocks meet two.
+    """
+    nb = n_blocks(n, block)
+    s = (n - 1) % block
+    col = np.zeros(nb, dtype=bool)
+    col[np.asarray(s_v, dtype=np.int64)] = True
+    col[0] = True
+    on = np.zeros(nb, dtype=bool)
+    on[np.asarray(s_s, dtype=np.int64)] = True
+    on[nb - 1] = True
+    csum = np.concatenate([[0], np.cumsum(on)])          # csum[i] = #selected in [0, i)
+    size = np.minimum(block, n - block * np.arange(nb))
+    qb = np.arange(nb)[:, None]
+    kb = np.arange(nb)[None, :]
+    dlt = qb - kb
+    vmin = -(size[:, None] - 1) + 0 * kb
+    vmax = np.where(dlt >= 1, size[None, :] - 1 + 0 * qb, 0)
+    lo = np.clip(nb - 1 - dlt + np.floor_divide(s + vmin, block), 0, nb)
+    hi = np.clip(nb - 1 - dlt + np.floor_divide(s + vmax, block), -1, nb - 1)
+    hit = (hi >= lo) & (csum[np.clip(hi + 1, 0, nb)] - csum[np.clip(lo, 0, nb)] > 0)
+    return (dlt >= 0) & (col[None, :] | hit)
+
+
 def vs_tile_mask_tokenwise(s_v, s_s, n: int, block: int) -> np.ndarray:
     """Brute-force definition of the same tile mask, token by token.
 
@@ -306,7 +366,7 @@ def vs_tile_mask_tokenwise(s_v, s_s, n: int, block: int) -> np.ndarray:
     vertical 0 and slash N_b-1 always kept). A tile is computed iff any of
     its (t, j) pairs is kept. O(n^2): small n only.
     """
-    nb = n // block
+    nb = n_blocks(n, block)
     cols = set(int(x) for x in s_v) | {0}
     slash = set(int(x) for x in s_s) | {nb - 1}
     mask = np.zeros((nb, nb), dtype=bool)
@@ -339,13 +399,14 @@ def masked_attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, tile_mask
     blocks (all when None). lse is the natural-log sum of exp of the logits.
     """
     n, d = q.shape
-    nb = n // block
+    nb = n_blocks(n, block)
     qbs = list(range(nb)) if qblocks is None else list(qblocks)
     outs, lses, rows = [], [], []
     for qb in qbs:
         kbs = np.nonzero(tile_mask[qb, : qb + 1])[0]
         keys = (kbs[:, None] * block + np.arange(block)[None, :]).reshape(-1)
-        t = qb * block + np.arange(block)
+        keys = keys[keys < n]
+        t = np.arange(qb * block, min(qb * block + block, n))
         z = (q[t] @ k[keys].T) * scale
         z = np.where(keys[None, :] <= t[:, None], z, -np.inf)
         m = z.max(axis=1, keepdims=True)
@@ -369,7 +430,7 @@ def head_route_and_select(q_head: np.ndarray, k_head: np.ndarray, prm: CrispPara
     """
     n, d = q_head.shape
     B = prm.block
-    nb = n // B
+    nb = n_blocks(n, B)
     scale = prm.scale(d)
     q_hat = q_head[n - B:]
     a_hat = proxy_attention(q_hat, k_head, scale)
@@ -400,7 +461,7 @@ def head_route_and_select(q_head: np.ndarray, k_head: np.ndarray, prm: CrispPara
         else:
             raise ValueError(f"unknown vs_rule {prm.vs_rule!r}")
         out["s_v"], out["s_s"] = s_v, s_s
-        out["mask"] = vs_tile_mask(s_v, s_s, nb)
+        out["mask"] = vs_tile_mask(s_v, s_s, nb, n, B)
     else:
         a_bar = pe_estimate(pe_pool(q_head, B), pe_pool(k_head, B), scale)
         sel = pe_index(a_bar, prm.gamma)
@@ -412,12 +473,15 @@ def head_route_and_select(q_head: np.ndarray, k_head: np.ndarray, prm: CrispPara
 
 def crisp_prefill(q, k, v, prm: CrispParams, qblocks: Optional[Sequence[int]] = None,
                   heads: Optional[Sequence[int]] = None, force_patterns: Optional[dict] = None,
-                  masks: Optional[dict] = None) -> Dict[str, object]:
+                  masks: Optional[dict] = None, lengths: Optional[Sequence[int]] = None
+                  ) -> Dict[str, object]:
     """Algorithm 1 over a whole [batch, H, n, d] problem (float64 numpy inputs).
 
     GQA: query head h reads KV head h // (H_q / H_kv). ``masks`` (keyed by
     (batch, head)) replaces the oracle's own tile masks for the attention
     step, so attention can be compared on another implementation's mask.
+    ``lengths`` gives each batch element's sequence length (its first
+    lengths[b] rows; the rest is padding the method never sees).
     Returns per (batch, head) dicts under "heads" and attention rows.
     """
     bsz, hq, n, d = q.shape
@@ -427,11 +491,12 @@ def crisp_prefill(q, k, v, prm: CrispParams, qblocks: Optional[Sequence[int]] = 
     res: Dict[str, object] = {"heads": {}, "attn": {}}
     heads = list(range(hq)) if heads is None else list(heads)
     for b in range(bsz):
+        nv = n if lengths is None else int(lengths[b])
         for h in heads:
             fp = None if force_patterns is None else force_patterns.get((b, h))
-            hr = head_route_and_select(q[b, h], k[b, h // g], prm, force_pattern=fp)
+            qh, kh, vh = q[b, h, :nv], k[b, h // g, :nv], v[b, h // g, :nv]
+            hr = head_route_and_select(qh, kh, prm, force_pattern=fp)
             res["heads"][(b, h)] = hr
             mask = hr["mask"] if masks is None else masks[(b, h)]
-            res["attn"][(b, h)] = masked_attention_rows(q[b, h], k[b, h // g], v[b, h // g],
-                                                        mask, prm.block, scale, qblocks)
+            res["attn"][(b, h)] = masked_attention_rows(qh, kh, vh, mask, prm.block, scale, qblocks)
     return res

@@ -18,6 +18,10 @@ adds exactly ``a*b`` to the scaled logit ``q.k/sqrt(dim)``):
   10000**(-k/8); ``"block"`` uses frequencies 2*pi*(k+1)/block, whose
   block sums are the same for every key block (no far-field structure).
 * diffuse heads: Q carries no planted component (near-uniform causal head).
+* variable lengths: with ``lengths`` set, batch element b is a sequence of
+  lengths[b] tokens stored in the first lengths[b] rows of its [seqlen, d]
+  slices (verticals drawn inside it); the remaining rows are padding,
+  filled with large finite values (N(0,1) * 64) that the method must ignore.
 
 Seeds: every (tensor, batch, head) slice has its own generator seeded from
 ``numpy.random.SeedSequence``; planted positions and per-head amplitudes
@@ -58,10 +62,15 @@ class Workload:
     recency_freqs: str = "block"
     v_unit: bool = False      # V ~ N(0,1) instead of N(0,1)/sqrt(dim)
     seed: int = 0
+    lengths: Optional[Sequence[int]] = None   # per-batch sequence lengths (<= seqlen)
 
     @property
     def n_blocks(self) -> int:
-        return self.seqlen // self.block
+        """Blocks of the longest sequence, ceil(seqlen / block)."""
+        return -(-self.seqlen // self.block)
+
+    def length(self, b: int) -> int:
+        return self.seqlen if self.lengths is None else int(self.lengths[b])
 
     def with_(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -102,9 +111,10 @@ def head_kinds(w: Workload) -> Dict[str, object]:
     else:
         sink = [float(w.sink_logit)] * w.h_q
     verticals: List[List[int]] = []
-    for _ in range(w.batch * w.h_kv):
+    for i in range(w.batch * w.h_kv):
         if w.n_vertical:
-            verticals.append(sorted(int(x) for x in rng.integers(w.block, w.seqlen - w.block,
+            n_b = w.length(i // w.h_kv)
+            verticals.append(sorted(int(x) for x in rng.integers(w.block, n_b - w.block,
                                                                    size=w.n_vertical)))
         else:
             verticals.append([])
@@ -154,6 +164,14 @@ def make_qkv(w: Workload, device: str = "cpu", heads_q: Optional[Sequence[int]] 
     q = torch.empty((w.batch, len(hq_list), N, d), dtype=torch.bfloat16, device=device)
     k = torch.empty((w.batch, w.h_kv, N, d), dtype=torch.bfloat16, device=device)
     v = torch.empty((w.batch, w.h_kv, N, d), dtype=torch.bfloat16, device=device)
+
+    def pad(x: torch.Tensor, tag: int, b: int, h: int) -> torch.Tensor:
+        n_b = w.length(b)
+        if n_b < N:
+            gen = torch.Generator(device=device)
+            gen.manual_seed(_slice_seed(w.seed, tag, b, h))
+            x[n_b:] = torch.randn((N - n_b, d), generator=gen, device=device, dtype=torch.float32) * 64.0
+        return x
     for b in range(w.batch):
         for hk in range(w.h_kv):
             x = randn(1, b, hk).mul_(inv)
@@ -163,11 +181,11 @@ def make_qkv(w: Workload, device: str = "cpu", heads_q: Optional[Sequence[int]] 
                 x[p, VERT_DIM] += 3.0 * c4
             if rope is not None:
                 x[:, :16] += rope
-            k[b, hk] = x.to(torch.bfloat16)
+            k[b, hk] = pad(x, 11, b, hk).to(torch.bfloat16)
             x = randn(2, b, hk)
             if not w.v_unit:
                 x.mul_(inv)
-            v[b, hk] = x.to(torch.bfloat16)
+            v[b, hk] = pad(x, 12, b, hk).to(torch.bfloat16)
         for i, h in enumerate(hq_list):
             x = randn(0, b, h).mul_(inv)
             if h not in diffuse:
@@ -176,7 +194,7 @@ def make_qkv(w: Workload, device: str = "cpu", heads_q: Optional[Sequence[int]] 
                     x[:, VERT_DIM] += 2.0 * c4
                 if rope is not None:
                     x[:, :16] += rope
-            q[b, i] = x.to(torch.bfloat16)
+            q[b, i] = pad(x, 10, b, h).to(torch.bfloat16)
     meta = dict(meta)
     meta["group"] = g
     return q, k, v, meta

@@ -372,6 +372,71 @@ def test_vs_tile_mask_matches_tokenwise_definition():
         np.testing.assert_array_equal(a, b)
 
 
+# --------------------------------------------------------------------------- ragged n
+# Section 4.3 partitions the map into N_b = ceil(n / B) blocks; the pins below
+# take n that is not a multiple of B (partial last block).
+RAGGED_N = [(8, 3 * 8 + 1), (8, 5 * 8 + 3), (8, 6 * 8 + 7), (4, 7 * 4 + 2), (16, 4 * 16 + 9)]
+
+
+def test_ragged_block_scores_bruteforce():
+    rng = _rng(21)
+    for B, n in RAGGED_N:
+        nb = -(-n // B)
+        assert O.n_blocks(n, B) == nb
+        q_hat, k = rng.standard_normal((B, 4)), rng.standard_normal((n, 4))
+        a = _proxy_bruteforce(q_hat.tolist(), k.tolist(), 0.8)
+        want_v, want_s = [0.0] * nb, [0.0] * nb
+        for r in range(B):
+            t = n - B + r
+            for j in range(t + 1):
+                want_v[j // B] += a[r][j] / B
+                want_s[(n - 1 - (t - j)) // B] += a[r][j] / B
+        p_v, p_s = O.vertical_slash_scores(O.proxy_attention(q_hat, k, 0.8), B)
+        assert p_v.shape == (nb,) and p_s.shape == (nb,)
+        np.testing.assert_allclose(p_v, want_v, atol=1e-14)
+        np.testing.assert_allclose(p_s, want_s, atol=1e-14)
+        np.testing.assert_allclose([p_v.sum(), p_s.sum()], [1.0, 1.0], atol=1e-13)
+        # the anchors of Eq. 2 are the first block and the (partial) last block
+        c = O.c_struct_from_map(O.proxy_attention(q_hat, k, 0.8), B)
+        last = sum(a[r][j] for r in range(B) for j in range((nb - 1) * B, n)) / B
+        first = sum(a[r][j] for r in range(B) for j in range(B)) / B
+        assert abs(c - (first + last)) < 1e-13
+
+
+def test_ragged_pooling_means_partial_block():
+    x = np.arange(22, dtype=np.float64).reshape(11, 2)        # 11 rows, B = 4: 4 + 4 + 3
+    pooled = O.pe_pool(x, 4)
+    assert pooled.shape == (3, 2)
+    np.testing.assert_array_equal(pooled[2], [(16 + 18 + 20) / 3, (17 + 19 + 21) / 3])
+    np.testing.assert_array_equal(pooled[0], [3.0, 4.0])
+
+
+def test_ragged_vs_tile_mask_matches_tokenwise_definition():
+    rng = _rng(22)
+    for B in (4, 8):
+        for n in [B * m + s for m in (3, 4, 7) for s in range(1, B)]:
+            nb = -(-n // B)
+            for _ in range(4):
+                s_v = rng.choice(nb, size=int(rng.integers(0, nb)), replace=False)
+                s_s = rng.choice(nb, size=int(rng.integers(0, nb)), replace=False)
+                a = O.vs_tile_mask(s_v, s_s, nb, n, B)
+                b = O.vs_tile_mask_tokenwise(s_v, s_s, n, B)
+                np.testing.assert_array_equal(a, b, err_msg=f"B={B} n={n}")
+
+
+def test_ragged_slash_block_can_meet_three_tile_diagonals():
+    # n = 8*8 + 3 (B = 8): slash block 3 holds slash indices 24..31, i.e. query-key
+    # offsets n-1-j* = 35..42, which tiles on diagonals 4 ([25, 39]), 5 ([33, 47])
+    # and 6 ([41, 55]) all contain; with n a multiple of B it would meet two.
+    B, n, nb = 8, 67, 9
+    m = O.vs_tile_mask([], [3], nb, n, B)
+    diags = sorted({qb - kb for qb in range(nb) for kb in range(1, qb + 1) if m[qb, kb] and qb - kb > 1})
+    assert diags == [4, 5, 6], diags
+    m2 = O.vs_tile_mask([], [3], 8, 64, B)
+    diags2 = sorted({qb - kb for qb in range(8) for kb in range(1, qb + 1) if m2[qb, kb] and qb - kb > 1})
+    assert diags2 == [4, 5], diags2
+
+
 # --------------------------------------------------------------------------- attention
 def _attention_bruteforce(q, k, v, allowed, scale):
     n, d = len(q), len(q[0])
@@ -411,6 +476,38 @@ def test_full_mask_equals_dense_causal_softmax():
     p /= p.sum(axis=1, keepdims=True)
     np.testing.assert_allclose(p.sum(axis=1), 1.0, atol=1e-14)
     np.testing.assert_allclose(o, p @ v, atol=1e-13)
+
+
+def test_ragged_full_mask_equals_dense_causal_softmax():
+    rng = _rng(23)
+    B = 8
+    for n in (27, 33, 47):
+        q, k, v = rng.standard_normal((3, n, 5))
+        nb = -(-n // B)
+        o, lse, rows = O.masked_attention_rows(q, k, v, np.tril(np.ones((nb, nb), dtype=bool)), B, 0.5)
+        want_o, want_lse = _attention_bruteforce(q.tolist(), k.tolist(), v.tolist(), lambda t, j: j <= t, 0.5)
+        assert rows.tolist() == list(range(n))
+        np.testing.assert_allclose(o, want_o, atol=1e-13)
+        np.testing.assert_allclose(lse, want_lse, atol=1e-13)
+
+
+def test_prefill_lengths_ignore_padding():
+    rng = _rng(24)
+    B, N = 8, 48
+    q, k, v = rng.standard_normal((3, 2, 2, N, 4))
+    lengths = [41, 30]
+    prm = O.CrispParams(block=B, k_min_blocks=1)
+    res = O.crisp_prefill(q, k, v, prm, lengths=lengths)
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    for b, nv in enumerate(lengths):               # padding rows change: nothing else may
+        q2[b, :, nv:] = 1e3
+        k2[b, :, nv:] = -1e3
+        v2[b, :, nv:] = 7.0
+    res2 = O.crisp_prefill(q2, k2, v2, prm, lengths=lengths)
+    for key, hr in res["heads"].items():
+        np.testing.assert_array_equal(hr["mask"], res2["heads"][key]["mask"])
+        np.testing.assert_array_equal(res["attn"][key][0], res2["attn"][key][0])
+        assert res["attn"][key][0].shape[0] == lengths[key[0]]
 
 
 def test_attention_is_causal():
