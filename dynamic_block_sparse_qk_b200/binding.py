@@ -42,19 +42,30 @@ class CrispParams(ctypes.Structure):
                 ("seqlen", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("block", ctypes.c_int32),
                 ("alpha", ctypes.c_float), ("gamma", ctypes.c_float), ("tau_proxy", ctypes.c_float),
                 ("tau_jsd", ctypes.c_float), ("k_min_blocks", ctypes.c_int32),
-                ("router", ctypes.c_int32), ("vs_rule", ctypes.c_int32), ("sm_scale", ctypes.c_float)]
+                ("router", ctypes.c_int32), ("vs_rule", ctypes.c_int32), ("sm_scale", ctypes.c_float),
+                ("seq_lens", ctypes.c_void_p)]
 
     @property
     def n_blocks(self) -> int:
-        return self.seqlen // self.block
+        """Blocks of the longest sequence (the stride of per-block outputs)."""
+        return -(-self.seqlen // self.block)
 
 
 def make_params(batch, h_q, h_kv, seqlen, head_dim, block=128, alpha=1.0, gamma=0.95,
                 tau_proxy=0.2, tau_jsd=0.1, k_min_blocks=8, router="cstruct", vs_rule="alpha",
-                sm_scale=0.0) -> CrispParams:
-    return CrispParams(batch, h_q, h_kv, seqlen, head_dim, block, alpha, gamma, tau_proxy, tau_jsd,
-                       k_min_blocks, ROUTER[router] if isinstance(router, str) else int(router),
-                       VS_RULE[vs_rule] if isinstance(vs_rule, str) else int(vs_rule), sm_scale)
+                sm_scale=0.0, seq_lens: Optional[torch.Tensor] = None) -> CrispParams:
+    """seq_lens: optional CUDA int32 tensor [batch] of sequence lengths. The
+    params keep only its device address: keep the tensor alive while they are
+    in use."""
+    if seq_lens is not None:
+        if not (seq_lens.is_cuda and seq_lens.dtype == torch.int32 and seq_lens.is_contiguous()
+                and seq_lens.numel() == batch):
+            raise ValueError("seq_lens must be a contiguous CUDA int32 tensor with one entry per batch element")
+    p = CrispParams(batch, h_q, h_kv, seqlen, head_dim, block, alpha, gamma, tau_proxy, tau_jsd,
+                    k_min_blocks, ROUTER[router] if isinstance(router, str) else int(router),
+                    VS_RULE[vs_rule] if isinstance(vs_rule, str) else int(vs_rule), sm_scale,
+                    None if seq_lens is None else seq_lens.data_ptr())
+    return p
 
 
 def params_for(q: torch.Tensor, k: torch.Tensor, **kw) -> CrispParams:

@@ -17,8 +17,7 @@ int check_params(const crisp_params* p) {
   if (p->h_q % p->h_kv) return CRISP_ERR_SHAPE;
   if (p->head_dim != 64 && p->head_dim != 128) return CRISP_ERR_SHAPE;
   if (p->block != 64 && p->block != 128) return CRISP_ERR_SHAPE;
-  if (p->seqlen % 128) return CRISP_ERR_SHAPE;
-  const long long nb = p->seqlen / p->block;
+  const long long nb = (static_cast<long long>(p->seqlen) + p->block - 1) / p->block;
   if (nb < 3 || nb > kMaxBlocks) return CRISP_ERR_SHAPE;
   // the PE softmax partials (ceil(N_b/64) per row) live in a [.][N_b][block] region
   if ((nb + 63) / 64 > p->block) return CRISP_ERR_SHAPE;
@@ -50,7 +49,7 @@ int to_status(cudaError_t e) { return e == cudaSuccess ? CRISP_OK : CRISP_ERR_CU
 
 extern "C" {
 
-int crisp_version(void) { return 10000; }
+int crisp_version(void) { return 10100; }
 
 const char* crisp_status_string(int s) {
   switch (s) {
@@ -102,7 +101,7 @@ int crisp_select(const crisp_params* p, const void* q, const void* k, const int3
   cudaError_t e = run_select(*p, q, k, pattern, p_v, p_s, ws, mask, tile_idx, tile_cnt, st);
   if (e == cudaSuccess && vs_sel) {
     const Workspace W = make_workspace(*p);
-    const size_t bytes = size_t(p->batch) * p->h_q * 2 * (p->seqlen / p->block);
+    const size_t bytes = size_t(p->batch) * p->h_q * 2 * n_blocks(*p);
     e = cudaMemcpyAsync(vs_sel, ws_ptr<char>(ws, W.sel), bytes, cudaMemcpyDeviceToDevice, st);
   }
   return to_status(e);

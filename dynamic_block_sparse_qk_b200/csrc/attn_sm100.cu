@@ -92,6 +92,7 @@ struct StepIter {
       for (int i = 0; i < 2; ++i) {
         if (i >= nsub) break;
         const int qb = qb0 + i;
+        if (qb >= nb) break;                 // a 64-wide block past the stored rows
         lst[i] = tile_idx + (size_t(bh) * nb + qb) * nb;
         int c = tile_cnt[size_t(bh) * nb + qb];
         if (c < 0 || c > qb + 1) {
@@ -184,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const Workspace W = make_workspace(p);
   int32_t* status = ws_ptr<int32_t>(ws, W.status);
-  const int N = p.seqlen, nb = N / p.block, NT = N / BM;
+  const int N = p.seqlen, nb = n_blocks(p), NT = (N + BM - 1) / BM;
   // Work order: KV-head major (the CTAs running at the same time read the same
   // K/V stream, which then stays in L2), longest query tiles first inside.
   const int g = p.h_q / p.h_kv;
@@ -198,6 +199,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int q_row = bh * N + row0;
   const int kv_row0 = (b * p.h_kv + hk) * N;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // This sequence's length: a query tile wholly past it only writes its
+  // stored rows as zeros (lse -inf).
+  const int len = seq_len(p, b, (qt == 0 && h == 0 && threadIdx.x == 0) ? status : nullptr);
+  if (row0 >= len) {
+    const int rows = min(BM, N - row0);
+    for (int i = threadIdx.x; i < rows * (D / 8); i += kThreads)
+      reinterpret_cast<uint4*>(o + (size_t(bh) * N + row0) * D)[i] = make_uint4(0, 0, 0, 0);
+    if (lse)
+      for (int i = threadIdx.x; i < rows; i += kThreads) lse[size_t(bh) * N + row0 + i] = -INFINITY;
+    return;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(C::B_Q), 1);
@@ -468,7 +480,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float w1 = l1 > 0.f ? fast_exp2(m1 - mm) : 0.f;
     const float lt = l0 * w0 + l1 * w1;
     __nv_bfloat16* orow = o + (size_t(bh) * N + row) * D + grp * (D / 2);
-    const bool fin = __all_sync(0xffffffffu, done && lt > 0.f);
+    // rows past the sequence (padding, or the next head's rows when the tile
+    // runs past seqlen) never decide the warp's path; stored padding rows are zero
+    const bool mine = row < len, stored = row < N;
+    const bool fin = __all_sync(0xffffffffu, done && (!mine || lt > 0.f));
     if (fin) {
       tc_fence_after();
       const float a0 = w0 / lt, a1 = w1 / lt;
@@ -488,16 +503,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float x1 = a1 != 0.f ? __uint_as_float(v1[q4 * 8 + e]) * a1 : 0.f;
             f[e] = x0 + x1;
           }
-          uint4 pk;
-          pk.x = pack_bf16(f[0], f[1]);
-          pk.y = pack_bf16(f[2], f[3]);
-          pk.z = pack_bf16(f[4], f[5]);
-          pk.w = pack_bf16(f[6], f[7]);
-          *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) = pk;
+          uint4 pk = make_uint4(0, 0, 0, 0);
+          if (mine) {
+            pk.x = pack_bf16(f[0], f[1]);
+            pk.y = pack_bf16(f[2], f[3]);
+            pk.z = pack_bf16(f[4], f[5]);
+            pk.w = pack_bf16(f[6], f[7]);
+          }
+          if (stored) *reinterpret_cast<uint4*>(orow + c * 32 + q4 * 8) = pk;
         }
       }
-      if (lse && grp == 0) lse[size_t(bh) * N + row] = (mm + log2f(lt)) * kLn2;
-    } else {
+      if (lse && grp == 0 && stored) lse[size_t(bh) * N + row] = mine ? (mm + log2f(lt)) * kLn2 : -INFINITY;
+    } else if (stored) {
       for (int c = 0; c < D / 2; c += 8) *reinterpret_cast<uint4*>(orow + c) = make_uint4(0, 0, 0, 0);
       if (lse && grp == 0) lse[size_t(bh) * N + row] = -INFINITY;
     }
@@ -525,7 +542,7 @@ cudaError_t launch_tc(const crisp_params& p, const void* q, const void* k, const
   auto kern = attn_tc_kernel<D, BLK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM);
   if (e != cudaSuccess) return e;
-  const unsigned grid = unsigned(p.batch) * p.h_q * (p.seqlen / BM);
+  const unsigned grid = unsigned(p.batch) * p.h_q * ((p.seqlen + BM - 1) / BM);
   kern<<<grid, kThreads, Cfg<D>::SMEM, st>>>(mq, mk, mv, tile_idx, tile_cnt, static_cast<__nv_bfloat16*>(o),
                                              lse, p, ws);
   return cudaGetLastError();

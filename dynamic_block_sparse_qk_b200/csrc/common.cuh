@@ -46,11 +46,30 @@ struct PeState {
   double above_sum;    // sum of entries strictly above the decided range
 };
 
+// Blocks of the longest sequence: N_b = ceil(seqlen / block) (the storage
+// stride of every per-block array).
+__host__ __device__ inline int n_blocks(const crisp_params& p) { return (p.seqlen + p.block - 1) / p.block; }
+
+// Length of sequence b: seq_lens[b] clamped to (2 * block, seqlen], or
+// seqlen without a length array. `status` (may be NULL) records a length
+// outside that range as CRISP_ERR_DEVICE.
+__device__ inline void report_error(int32_t* status, int32_t code, int32_t where);
+__device__ inline int seq_len(const crisp_params& p, int b, int32_t* status = nullptr) {
+  if (!p.seq_lens) return p.seqlen;
+  const int n = p.seq_lens[b];
+  const int lo = 2 * p.block + 1;
+  if (n < lo || n > p.seqlen) {
+    if (status) report_error(status, CRISP_ERR_DEVICE, n);
+    return n < lo ? lo : p.seqlen;
+  }
+  return n;
+}
+
 // Key tiles per proxy CTA: small enough that short sequences still give about
 // four CTAs per SM (148 SMs), at most 32 for long ones; even, so a 128-key
 // step of 64-wide blocks never straddles two chunks.
 __host__ __device__ inline int proxy_chunk(const crisp_params& p) {
-  const long long nb = p.seqlen / p.block;
+  const long long nb = n_blocks(p);
   long long c = (nb * p.batch * p.h_q + 591) / 592;
   c = c < 4 ? 4 : (c > 32 ? 32 : c);
   return int((c + 1) & ~1ll);
@@ -64,7 +83,7 @@ __host__ __device__ inline Workspace make_workspace(const crisp_params& p) {
   Workspace w{};
   const size_t BH = size_t(p.batch) * p.h_q;
   const size_t BK = size_t(p.batch) * p.h_kv;
-  const size_t nb = size_t(p.seqlen / p.block);
+  const size_t nb = size_t(n_blocks(p));
   const size_t R = size_t(p.block);
   const size_t nc = (nb + proxy_chunk(p) - 1) / proxy_chunk(p);
   const size_t d = size_t(p.head_dim);

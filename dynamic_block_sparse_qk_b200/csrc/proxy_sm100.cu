@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(kPxThreads, 2)
 
   const Workspace W = make_workspace(p);
   int32_t* status = ws_ptr<int32_t>(ws, W.status);
-  const int N = p.seqlen, nb = N / R;
+  const int N = p.seqlen, nb = n_blocks(p);
   const int chunk_tiles = proxy_chunk(p);
   const int nc = (nb + chunk_tiles - 1) / chunk_tiles;
   // CTA order: the query heads of one KV head are adjacent, so the CTAs that
@@ -104,9 +104,12 @@ __global__ void __launch_bounds__(kPxThreads, 2)
   const int chunk = t % nc, bk = t / nc;          // bk = batch * h_kv + kv head
   const int b = bk / p.h_kv, hk = bk % p.h_kv;
   const int bh = b * p.h_q + hk * g + hin;
-  const int kb0 = chunk * chunk_tiles, kb1 = min(kb0 + chunk_tiles, nb);
-  const int nsteps = (kb1 - kb0 + KPS - 1) / KPS;
-  const int q_row = bh * N + N - PM;
+  // this sequence's length and blocks (chunks past its end have no steps)
+  const int len = seq_len(p, b, (chunk == 0 && hin == 0 && hk == 0 && threadIdx.x == 0) ? status : nullptr);
+  const int nbv = (len + R - 1) / R;
+  const int kb0 = chunk * chunk_tiles, kb1 = min(kb0 + chunk_tiles, nbv);
+  const int nsteps = kb1 > kb0 ? (kb1 - kb0 + KPS - 1) / KPS : 0;
+  const int q_row = bh * N + len - PM;
   const int k_row0 = bk * N + kb0 * R;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -201,9 +204,24 @@ __global__ void __launch_bounds__(kPxThreads, 2)
 
     // exp2(s * sl2 - mx) summed over one 32-column chunk into lo (columns <= pr)
     // and hi (columns > pr); `ci` is the chunk index inside its key tile.
-    auto chunk_sums = [&](const uint32_t (&a)[32], int ci, bool last, float mx, uint64_t& lo2, uint64_t& hi2) {
+    // `lim` is the last key column this row may see in the tile (causal
+    // limit); only the last two tiles of a sequence (`masked`) have one below
+    // the tile width, and there every column is tested on its own.
+    auto chunk_sums = [&](const uint32_t (&a)[32], int ci, bool masked, int lim, float mx, uint64_t& lo2,
+                          uint64_t& hi2) {
       const uint64_t nm2 = pack_f32x2(-mx, -mx);
-      if (ci < mixc || (ci > mixc && !last)) {
+      if (masked) {
+        float lo = 0.f, hi = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c = ci * 32 + e;
+          const float ex = c <= lim ? fast_exp2(fmaf(__uint_as_float(a[e]), sl2, -mx)) : 0.f;
+          if (c <= pr) lo += ex;
+          else hi += ex;
+        }
+        lo2 = add_f32x2(lo2, pack_f32x2(lo, 0.f));
+        hi2 = add_f32x2(hi2, pack_f32x2(hi, 0.f));
+      } else if (ci != mixc) {
         uint64_t acc2[2] = {pack_f32x2(0.f, 0.f), pack_f32x2(0.f, 0.f)};
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
@@ -215,7 +233,7 @@ __global__ void __launch_bounds__(kPxThreads, 2)
         const uint64_t sum2 = add_f32x2(acc2[0], acc2[1]);
         if (ci < mixc) lo2 = add_f32x2(lo2, sum2);
         else hi2 = add_f32x2(hi2, sum2);
-      } else if (ci == mixc) {
+      } else {
         float lo = 0.f, hi = 0.f;
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
@@ -224,38 +242,42 @@ __global__ void __launch_bounds__(kPxThreads, 2)
           else hi += ex;
         }
         lo2 = add_f32x2(lo2, pack_f32x2(lo, 0.f));
-        if (!last) hi2 = add_f32x2(hi2, pack_f32x2(hi, 0.f));
+        hi2 = add_f32x2(hi2, pack_f32x2(hi, 0.f));
       }
     };
-    // max over one chunk (raw scores); on the last key tile only columns <= pr count
-    auto chunk_max = [&](const uint32_t (&a)[32], int ci, bool last, float mx) -> float {
-      if (!last || ci < mixc) {
+    // max over one chunk (raw scores), visible columns only
+    auto chunk_max = [&](const uint32_t (&a)[32], int ci, bool masked, int lim, float mx) -> float {
+      if (!masked) {
         float m2[2] = {mx, -INFINITY};
 #pragma unroll
         for (int e = 0; e < 32; e += 2)
           m2[(e >> 1) & 1] = max3f(m2[(e >> 1) & 1], __uint_as_float(a[e]), __uint_as_float(a[e + 1]));
         return fmaxf(m2[0], m2[1]);
       }
-      if (ci == mixc) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (e <= prl) mx = fmaxf(mx, __uint_as_float(a[e]));
-      }
+      for (int e = 0; e < 32; ++e)
+        if (ci * 32 + e <= lim) mx = fmaxf(mx, __uint_as_float(a[e]));
       return mx;
     };
-    auto finish_tile = [&](int kb, bool last, float mx, uint64_t lo2, uint64_t hi2) {
+    // A row with no visible key in the tile (possible in a partial last block)
+    // stores max -inf and zero sums and leaves the running (max, sum) alone.
+    auto finish_tile = [&](int kb, float mx, uint64_t lo2, uint64_t hi2) {
       float l0, l1, h0, h1;
       unpack_f32x2(lo2, l0, l1);
       unpack_f32x2(hi2, h0, h1);
-      const float lo = l0 + l1, hi = last ? 0.f : h0 + h1;
+      const bool any = mx != -INFINITY;
+      const float lo = any ? l0 + l1 : 0.f, hi = any ? h0 + h1 : 0.f;
       const size_t o = (size_t(bh) * nb + kb) * R + pr;
       stat_m[o] = mx;
       stat_lo[o] = lo;
       stat_hi[o] = hi;
-      const float nm = fmaxf(cm, mx);
-      cl = cl * fast_exp2(cm - nm) + (lo + hi) * fast_exp2(mx - nm);
-      cm = nm;
+      if (any) {
+        const float nm = fmaxf(cm, mx);
+        cl = cl * fast_exp2(cm - nm) + (lo + hi) * fast_exp2(mx - nm);
+        cm = nm;
+      }
     };
+    const int t_row = len - R + pr;            // position of this proxy row
 
     int u = 0;
     for (int j = grp; j < nsteps; j += 2, ++u) {
@@ -278,42 +300,51 @@ __global__ void __launch_bounds__(kPxThreads, 2)
           }
           const int kb = kbs + ks;
           if (kb < kb1) {
-            const bool last = kb == nb - 1;
-            float mx = chunk_max(a0, 0, last, -INFINITY);
-            mx = chunk_max(a1, 1, last, mx) * sl2;
+            const bool masked = kb >= nbv - 2;
+            const int lim = t_row - kb * R;
+            float mx = chunk_max(a0, 0, masked, lim, -INFINITY);
+            mx = chunk_max(a1, 1, masked, lim, mx) * sl2;
             uint64_t lo2 = pack_f32x2(0.f, 0.f), hi2 = pack_f32x2(0.f, 0.f);
-            chunk_sums(a0, 0, last, mx, lo2, hi2);
-            chunk_sums(a1, 1, last, mx, lo2, hi2);
-            finish_tile(kb, last, mx, lo2, hi2);
+            if (mx != -INFINITY) {
+              chunk_sums(a0, 0, masked, lim, mx, lo2, hi2);
+              chunk_sums(a1, 1, masked, lim, mx, lo2, hi2);
+            }
+            finish_tile(kb, mx, lo2, hi2);
           }
         }
       } else {
         // one 128-key tile: a max pass and a sum pass over two pairs of chunks
         const int kb = kbs;
-        const bool last = kb == nb - 1;
+        const bool masked = kb >= nbv - 2;
+        const int lim = t_row - kb * R;
         tmem_ld32(tS, a0);
         tmem_ld32(tS + 32, a1);
         tmem_wait_ld();
-        float mx = chunk_max(a0, 0, last, -INFINITY);
-        mx = chunk_max(a1, 1, last, mx);
+        float mx = chunk_max(a0, 0, masked, lim, -INFINITY);
+        mx = chunk_max(a1, 1, masked, lim, mx);
         uint32_t a2[32], a3[32];
         tmem_ld32(tS + 64, a2);
         tmem_ld32(tS + 96, a3);
         tmem_wait_ld();
-        mx = chunk_max(a2, 2, last, mx);
-        mx = chunk_max(a3, 3, last, mx) * sl2;
+        mx = chunk_max(a2, 2, masked, lim, mx);
+        mx = chunk_max(a3, 3, masked, lim, mx) * sl2;
         uint64_t lo2 = pack_f32x2(0.f, 0.f), hi2 = pack_f32x2(0.f, 0.f);
-        chunk_sums(a2, 2, last, mx, lo2, hi2);
-        chunk_sums(a3, 3, last, mx, lo2, hi2);
+        const bool any = mx != -INFINITY;
+        if (any) {
+          chunk_sums(a2, 2, masked, lim, mx, lo2, hi2);
+          chunk_sums(a3, 3, masked, lim, mx, lo2, hi2);
+        }
         tmem_ld32(tS, a0);
         tmem_ld32(tS + 32, a1);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::B_SFREE + grp));
-        chunk_sums(a0, 0, last, mx, lo2, hi2);
-        chunk_sums(a1, 1, last, mx, lo2, hi2);
-        finish_tile(kb, last, mx, lo2, hi2);
+        if (any) {
+          chunk_sums(a0, 0, masked, lim, mx, lo2, hi2);
+          chunk_sums(a1, 1, masked, lim, mx, lo2, hi2);
+        }
+        finish_tile(kb, mx, lo2, hi2);
       }
     }
     // ---- merge the two groups' running (max, sum) for this chunk (every
@@ -372,7 +403,7 @@ cudaError_t launch_proxy(const crisp_params& p, const void* q, const void* k, vo
   auto kern = proxy_tc_kernel<D, R>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PxCfg<D>::SMEM);
   if (e != cudaSuccess) return e;
-  const int nb = p.seqlen / R;
+  const int nb = n_blocks(p);
   const int nc = (nb + proxy_chunk(p) - 1) / proxy_chunk(p);
   const unsigned grid = unsigned(p.batch) * p.h_q * nc;
   kern<<<grid, kPxThreads, PxCfg<D>::SMEM, st>>>(mq, mk, p, ws);

@@ -25,11 +25,16 @@ __global__ void proxy_scores_kernel(crisp_params p, void* ws, float* __restrict_
                                     float* __restrict__ score) {
   __shared__ int last;
   const Workspace W = make_workspace(p);
-  const int R = p.block, nb = p.seqlen / p.block;
+  const int R = p.block, nb = n_blocks(p);
   const int bh = blockIdx.y;
+  const int nbv = (seq_len(p, bh / p.h_q) + R - 1) / R;   // this sequence's blocks
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kb = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (kb < nb) {
+  if (kb >= nbv && kb < nb && lane == 0) {          // past the end of a shorter sequence
+    p_v[size_t(bh) * nb + kb] = 0.f;
+    p_s[size_t(bh) * nb + kb] = 0.f;
+  }
+  if (kb < nbv) {
     const float* sm = ws_ptr<float>(ws, W.stat_m) + size_t(bh) * nb * R;
     const float* slo = ws_ptr<float>(ws, W.stat_lo) + size_t(bh) * nb * R;
     const float* shi = ws_ptr<float>(ws, W.stat_hi) + size_t(bh) * nb * R;
@@ -62,7 +67,7 @@ __global__ void proxy_scores_kernel(crisp_params p, void* ws, float* __restrict_
   __syncthreads();
   if (!last || threadIdx.x != 0) return;
   __threadfence();
-  const float c = __ldcg(p_v + size_t(bh) * nb) + __ldcg(p_v + size_t(bh) * nb + nb - 1);
+  const float c = __ldcg(p_v + size_t(bh) * nb) + __ldcg(p_v + size_t(bh) * nb + nbv - 1);
   score[bh] = c;
   pattern[bh] = (c >= p.tau_proxy) ? CRISP_PATTERN_VS : CRISP_PATTERN_PE;
   *cnt = 0u;
@@ -83,10 +88,13 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   constexpr int CPR = D / 8;
   constexpr int RPP = 256 / CPR;   // rows per pass
   __shared__ float part[RPP][D];
-  const int R = p.block, nb = p.seqlen / p.block;
+  const int R = p.block, nb = n_blocks(p);
   const int kb = blockIdx.x;
   const bool is_k = int(blockIdx.y) < nk;
   const int hh = is_k ? int(blockIdx.y) : int(blockIdx.y) - nk;
+  const int len = seq_len(p, hh / (is_k ? p.h_kv : p.h_q));
+  const int rows = min(R, len - kb * R);            // a partial last block averages what it holds
+  if (rows <= 0) return;
   const __nv_bfloat16* x = is_k ? k : q;
   float* out = is_k ? kbar : qbar;
   if (pattern) {
@@ -103,7 +111,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   const int tid = threadIdx.x, c = tid % CPR, rg = tid / CPR;
   const __nv_bfloat16* src = x + (size_t(hh) * p.seqlen + size_t(kb) * R) * D;
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  for (int row = rg; row < R; row += RPP) {
+  for (int row = rg; row < rows; row += RPP) {
     const uint4 u = *reinterpret_cast<const uint4*>(src + size_t(row) * D + c * 8);
     const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
@@ -120,7 +128,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
     float s = 0.f;
 #pragma unroll
     for (int i = 0; i < RPP; ++i) s += part[i][dd];
-    out[(size_t(hh) * nb + kb) * D + dd] = s / float(R);
+    out[(size_t(hh) * nb + kb) * D + dd] = s / float(rows);
   }
 }
 
@@ -139,13 +147,15 @@ __global__ void __launch_bounds__(256) route_kernel(const __nv_bfloat16* __restr
   __shared__ float qm[D];
   __shared__ float red[32];
   const Workspace W = make_workspace(p);
-  const int nb = p.seqlen / p.block, R = p.block;
+  const int nb = n_blocks(p), R = p.block;
   const int bh = blockIdx.x;
+  const int len = seq_len(p, bh / p.h_q);
+  const int nbv = (len + R - 1) / R;              // this sequence's blocks
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const float* pv = p_v + size_t(bh) * nb;
   const float scale = p.sm_scale > 0.f ? p.sm_scale : rsqrtf(float(D));
   const size_t N = size_t(p.seqlen);
-  const __nv_bfloat16* qh = q + (size_t(bh) * N + N - R) * D;
+  const __nv_bfloat16* qh = q + (size_t(bh) * N + len - R) * D;
   for (int dd = tid; dd < D; dd += 256) {
     float s = 0.f;
     for (int r = 0; r < R; ++r) s += __bfloat162float(qh[size_t(r) * D + dd]);
@@ -156,7 +166,7 @@ __global__ void __launch_bounds__(256) route_kernel(const __nv_bfloat16* __restr
   const int hk = h / (p.h_q / p.h_kv);
   const float* kbar = ws_ptr<float>(ws, W.kbar) + (size_t(b) * p.h_kv + hk) * nb * D;
   float lmax = -INFINITY;
-  for (int kb = warp; kb < nb; kb += 8) {
+  for (int kb = warp; kb < nbv; kb += 8) {
     float s = 0.f;
     for (int dd = lane; dd < D; dd += 32) s += qm[dd] * kbar[size_t(kb) * D + dd];
     s = warp_sum(s) * scale;
@@ -169,7 +179,7 @@ __global__ void __launch_bounds__(256) route_kernel(const __nv_bfloat16* __restr
   for (int i = 0; i < 8; ++i) zmax = fmaxf(zmax, red[i]);
   __syncthreads();
   float lsum = 0.f;
-  for (int kb = tid; kb < nb; kb += 256) {
+  for (int kb = tid; kb < nbv; kb += 256) {
     const float e = expf(zs[kb] - zmax);
     zs[kb] = e;
     lsum += e;
@@ -182,7 +192,7 @@ __global__ void __launch_bounds__(256) route_kernel(const __nv_bfloat16* __restr
   __syncthreads();
   // KL(a_hat || m) + KL(a_bar || m), natural log, 0 log 0 = 0.
   float kl = 0.f;
-  for (int kb = tid; kb < nb; kb += 256) {
+  for (int kb = tid; kb < nbv; kb += 256) {
     const float ah = pv[kb], ab = zs[kb] / zsum;
     const float m = 0.5f * (ah + ab);
     if (ah > 0.f) kl += ah * logf(ah / m);
@@ -206,7 +216,7 @@ __global__ void __launch_bounds__(256) route_kernel(const __nv_bfloat16* __restr
 cudaError_t launch_pool(const crisp_params& p, const void* k, const void* q, int nk, int nq,
                         const int32_t* pattern, float* kbar, float* qbar, cudaStream_t st) {
   if (nk + nq == 0) return cudaSuccess;
-  const int nb = p.seqlen / p.block;
+  const int nb = n_blocks(p);
   dim3 grid(nb, nk + nq);
   const auto* kk = static_cast<const __nv_bfloat16*>(k);
   const auto* qq = static_cast<const __nv_bfloat16*>(q);
@@ -220,7 +230,7 @@ cudaError_t launch_pool(const crisp_params& p, const void* k, const void* q, int
 cudaError_t run_route(const crisp_params& p, const void* q, const void* k, void* ws,
                       int32_t* pattern, float* score, float* p_v, float* p_s, cudaStream_t st) {
   const Workspace W = make_workspace(p);
-  const int nb = p.seqlen / p.block;
+  const int nb = n_blocks(p);
   const int BH = p.batch * p.h_q;
   // proxy statistics (+ row merge in the last CTA of each head), block
   // scores (+ C_struct route in the last CTA of each head)

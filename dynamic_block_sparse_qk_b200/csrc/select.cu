@@ -19,17 +19,19 @@ __global__ void __launch_bounds__(1024) vs_select_kernel(crisp_params p, const i
                                                          const float* __restrict__ p_v,
                                                          const float* __restrict__ p_s, void* ws) {
   extern __shared__ unsigned char sm[];
-  const int nb = p.seqlen / p.block;
-  float* pv = reinterpret_cast<float*>(sm);                 // [nb]
-  float* sorted = pv + nb;                                   // [nb] (GAMMA)
-  double* scan = reinterpret_cast<double*>(sorted + nb);  // [1024], 8-byte aligned (2*nb floats)
+  const int nbs = n_blocks(p);                               // stride of the per-block arrays
+  float* pv = reinterpret_cast<float*>(sm);                 // [nbs]
+  float* sorted = pv + nbs;                                  // [nbs] (GAMMA)
+  double* scan = reinterpret_cast<double*>(sorted + nbs); // [1024], 8-byte aligned (2*nbs floats)
   __shared__ int cnt_s, kcut_s;
   __shared__ float med_s[2];
   const Workspace W = make_workspace(p);
   const int bh = blockIdx.x, dir = blockIdx.y;
-  const float* src = (dir == 0 ? p_v : p_s) + size_t(bh) * nb;
-  uint8_t* sel = ws_ptr<uint8_t>(ws, W.sel) + (size_t(bh) * 2 + dir) * nb;
+  const float* src = (dir == 0 ? p_v : p_s) + size_t(bh) * nbs;
+  uint8_t* sel = ws_ptr<uint8_t>(ws, W.sel) + (size_t(bh) * 2 + dir) * nbs;
   const int tid = threadIdx.x;
+  const int nb = (seq_len(p, bh / p.h_q) + p.block - 1) / p.block;   // this sequence's blocks
+  for (int j = nb + tid; j < nbs; j += 1024) sel[j] = 0;
   // Fresh state for this head's PE path, which runs after this kernel in
   // stream order: radix-select histograms (half per direction CTA), the cut
   // state and the completion counters of the histogram and tie kernels.
@@ -141,11 +143,12 @@ __global__ void __launch_bounds__(256) pe_logits_kernel(crisp_params p, const in
   __shared__ float kst[KC][T + 1];
   __shared__ float rmax[T][17], rsum[T][17];
   const Workspace W = make_workspace(p);
-  const int nb = p.seqlen / p.block;
+  const int nb = n_blocks(p);                               // stride
   const int bh = blockIdx.z;
   if (pattern[bh] != CRISP_PATTERN_PE) return;
+  const int nbv = (seq_len(p, bh / p.h_q) + p.block - 1) / p.block;   // this sequence's blocks
   const int tq = blockIdx.y, tk = blockIdx.x;
-  if (tk > tq) return;
+  if (tk > tq || tq * 64 >= nbv) return;
   const int b = bh / p.h_q, h = bh % p.h_q, hk = h / (p.h_q / p.h_kv);
   const float* qbar = ws_ptr<float>(ws, W.qbar) + size_t(bh) * nb * D;
   const float* kbar = ws_ptr<float>(ws, W.kbar) + (size_t(b) * p.h_kv + hk) * nb * D;
@@ -157,8 +160,8 @@ __global__ void __launch_bounds__(256) pe_logits_kernel(crisp_params p, const in
     for (int i = tid; i < T * KC; i += 256) {
       const int r = i / KC, c = i % KC;
       const int qr = tq * T + r, kr = tk * T + r;
-      qs[c][r] = qr < nb ? qbar[size_t(qr) * D + k0 + c] : 0.f;
-      kst[c][r] = kr < nb ? kbar[size_t(kr) * D + k0 + c] : 0.f;
+      qs[c][r] = qr < nbv ? qbar[size_t(qr) * D + k0 + c] : 0.f;
+      kst[c][r] = kr < nbv ? kbar[size_t(kr) * D + k0 + c] : 0.f;
     }
     __syncthreads();
 #pragma unroll 8
@@ -181,7 +184,7 @@ __global__ void __launch_bounds__(256) pe_logits_kernel(crisp_params p, const in
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int kb = tk * T + tx * 4 + j;
-      const bool ok = qb < nb && kb <= qb;
+      const bool ok = qb < nbv && kb <= qb;
       acc[i][j] = ok ? acc[i][j] * sl2 : -INFINITY;
       if (ok) abar[size_t(qb) * nb + kb] = acc[i][j];
       mx = fmaxf(mx, acc[i][j]);
@@ -195,7 +198,7 @@ __global__ void __launch_bounds__(256) pe_logits_kernel(crisp_params p, const in
   __syncthreads();
   if (tid < T) {
     const int qb = tq * T + tid;
-    if (qb < nb) {
+    if (qb < nbv) {
       float mx = -INFINITY;
       for (int j = 0; j < 16; ++j) mx = fmaxf(mx, rmax[tid][j]);
       float s = 0.f;
@@ -212,12 +215,13 @@ __global__ void __launch_bounds__(256) pe_logits_kernel(crisp_params p, const in
 // One warp per PE row: combine partials, rewrite abar[qb][kb] = softmax / N_b.
 __global__ void pe_normalize_kernel(crisp_params p, const int32_t* pattern, void* ws) {
   const Workspace W = make_workspace(p);
-  const int nb = p.seqlen / p.block;
+  const int nb = n_blocks(p);                               // stride
   const int bh = blockIdx.y;
   if (pattern[bh] != CRISP_PATTERN_PE) return;
+  const int nbv = (seq_len(p, bh / p.h_q) + p.block - 1) / p.block;   // this sequence's blocks
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qb = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (qb >= nb) return;
+  if (qb >= nbv) return;
   const int ntile = (nb + 63) / 64;
   const int nt = qb / 64 + 1;
   const float* pm = ws_ptr<float>(ws, W.stat_m) + (size_t(bh) * nb + qb) * ntile;
@@ -228,7 +232,7 @@ __global__ void pe_normalize_kernel(crisp_params p, const int32_t* pattern, void
   float s = 0.f;
   for (int t = lane; t < nt; t += 32) s += ps[t] * exp2f(pm[t] - mx);
   s = warp_sum(s);
-  const float inv = 1.0f / (s * float(nb));
+  const float inv = 1.0f / (s * float(nbv));               // Algorithm 4: the total is N_b
   float* row = ws_ptr<float>(ws, W.abar) + (size_t(bh) * nb + qb) * nb;
   for (int kb = lane; kb <= qb; kb += 32) row[kb] = exp2f(row[kb] - mx) * inv;
 }
@@ -311,18 +315,19 @@ __global__ void __launch_bounds__(256) pe_hist_kernel(crisp_params p, const int3
   __shared__ uint32_t hc[4096];
   __shared__ double hs[4096];
   const Workspace W = make_workspace(p);
-  const int nb = p.seqlen / p.block;
+  const int nb = n_blocks(p);                               // stride
   const int bh = blockIdx.y;
   if (pattern[bh] != CRISP_PATTERN_PE) return;
   const PeState st = ws_ptr<PeState>(ws, W.pe_state)[bh];
   if (st.all) return;
+  const int nbv = (seq_len(p, bh / p.h_q) + p.block - 1) / p.block;   // this sequence's blocks
   int shift, nbk;
   level_geom(level, shift, nbk);
   for (int i = threadIdx.x; i < nbk; i += 256) { hc[i] = 0; hs[i] = 0.0; }
   __syncthreads();
   const float* abar = ws_ptr<float>(ws, W.abar) + size_t(bh) * nb * nb;
   const int rows_per = 8;
-  const int q0 = blockIdx.x * rows_per, q1 = min(q0 + rows_per, nb);
+  const int q0 = blockIdx.x * rows_per, q1 = min(q0 + rows_per, nbv);
   const uint32_t hi_shift = shift + (level == 2 ? 8 : 12);
   // The entries of a row are close in value, so the lanes of a warp mostly hit
   // one or two buckets. Lanes with the same bucket combine first: each lane
@@ -390,17 +395,18 @@ __global__ void __launch_bounds__(256) pe_eqcount_kernel(crisp_params p, const i
   __shared__ uint32_t part[256];
   __shared__ int last;
   const Workspace W = make_workspace(p);
-  const int nb = p.seqlen / p.block;
+  const int nbs = n_blocks(p);                              // stride
   const int bh = blockIdx.y;
   if (pattern[bh] != CRISP_PATTERN_PE) return;
   const PeState st = ws_ptr<PeState>(ws, W.pe_state)[bh];
   if (st.all) return;
+  const int nb = (seq_len(p, bh / p.h_q) + p.block - 1) / p.block;    // this sequence's blocks
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qb = blockIdx.x * 8 + warp;
-  uint32_t* ec = ws_ptr<uint32_t>(ws, W.eq_cnt) + size_t(bh) * nb;
+  uint32_t* ec = ws_ptr<uint32_t>(ws, W.eq_cnt) + size_t(bh) * nbs;
   if (qb < nb) {
     const float tv = __uint_as_float(st.prefix);
-    const float* row = ws_ptr<float>(ws, W.abar) + (size_t(bh) * nb + qb) * nb;
+    const float* row = ws_ptr<float>(ws, W.abar) + (size_t(bh) * nbs + qb) * nbs;
     uint32_t c = 0;
     for (int kb = lane; kb <= qb; kb += 32) c += row[kb] == tv;
     c = __reduce_add_sync(0xffffffffu, c);
@@ -447,34 +453,56 @@ __global__ void __launch_bounds__(256) build_tiles_kernel(crisp_params p, const 
                                                           int32_t* __restrict__ tile_idx,
                                                           int32_t* __restrict__ tile_cnt) {
   const Workspace W = make_workspace(p);
-  const int nb = p.seqlen / p.block;
+  const int nbs = n_blocks(p);                              // stride of the per-block arrays
   const int bh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qb = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (qb >= nb) return;
+  if (qb >= nbs) return;
+  const int B = p.block;
+  const int len = seq_len(p, bh / p.h_q);
+  const int nb = (len + B - 1) / B;                         // this sequence's blocks
+  int32_t* idx = tile_idx + (size_t(bh) * nbs + qb) * nbs;
+  uint8_t* mrow = mask ? mask + (size_t(bh) * nbs + qb) * nbs : nullptr;
+  if (qb >= nb) {                                           // past the end of a shorter sequence
+    if (lane == 0) tile_cnt[size_t(bh) * nbs + qb] = 0;
+    for (int j = lane; mrow && j < nbs; j += 32) mrow[j] = 0;
+    return;
+  }
   const bool vs = pattern[bh] == CRISP_PATTERN_VS;
-  const uint8_t* sv = ws_ptr<uint8_t>(ws, W.sel) + size_t(bh) * 2 * nb;
-  const uint8_t* ss = sv + nb;
+  const uint8_t* sv = ws_ptr<uint8_t>(ws, W.sel) + size_t(bh) * 2 * nbs;
+  const uint8_t* ss = sv + nbs;
   PeState st{};
   const float* arow = nullptr;
   uint32_t eq_before = 0;
   float tv = 0.f;
   if (!vs) {
     st = ws_ptr<PeState>(ws, W.pe_state)[bh];
-    arow = ws_ptr<float>(ws, W.abar) + (size_t(bh) * nb + qb) * nb;
+    arow = ws_ptr<float>(ws, W.abar) + (size_t(bh) * nbs + qb) * nbs;
     tv = __uint_as_float(st.prefix);
-    if (!st.all) eq_before = ws_ptr<uint32_t>(ws, W.eq_cnt)[size_t(bh) * nb + qb];
+    if (!st.all) eq_before = ws_ptr<uint32_t>(ws, W.eq_cnt)[size_t(bh) * nbs + qb];
   }
-  auto offset_on = [&](int o) -> bool {
-    if (o == 0) return true;
-    if (o < 0 || o >= nb) return false;
-    return ss[nb - 1 - o] != 0;
+  // Slash blocks met by tile (qb, kb): pair (t, j) lies on slash index
+  // j + len-1-t = (nb-1-delta) B + s + (c - r) with s = (len-1) mod B and
+  // c - r over [-(rows(qb)-1), cols(kb)-1] (off the diagonal) or
+  // [-(rows(qb)-1), 0] (on it); so the blocks nb-1-delta + {-1, 0, +1}
+  // with the two ends decided by the signs below. For len a multiple of B
+  // this is {nb-1-delta, nb-delta}: offsets delta and delta-1.
+  const int s_res = (len - 1) % B;
+  const int rows_q = min(B, len - qb * B);
+  const bool lo_ext = s_res - (rows_q - 1) < 0;
+  auto slash_on = [&](int jb) -> bool { return jb == nb - 1 || (jb >= 0 && jb < nb && ss[jb] != 0); };
+  auto slash_hit = [&](int kb) -> bool {
+    const int dlt = qb - kb;
+    const int vmax = dlt >= 1 ? B - 1 : 0;                  // key blocks before qb are full
+    const int lo = nb - 1 - dlt - (lo_ext ? 1 : 0);
+    const int hi = nb - 1 - dlt + (s_res + vmax >= B ? 1 : 0);
+    for (int jb = lo; jb <= hi; ++jb)
+      if (slash_on(jb)) return true;
+    return false;
   };
-  int32_t* idx = tile_idx + (size_t(bh) * nb + qb) * nb;
-  uint8_t* mrow = mask ? mask + (size_t(bh) * nb + qb) * nb : nullptr;
   int count = 0;
   uint32_t eq_seen = eq_before;
-  for (int base = 0; base < nb; base += 128) {
+  for (int base = 0; base <= qb; base += 128) {
     bool f[4];
     int neq = 0;
     bool isq[4];
@@ -485,8 +513,7 @@ __global__ void __launch_bounds__(256) build_tiles_kernel(crisp_params p, const 
       isq[i] = false;
       if (kb <= qb) {
         if (vs) {
-          const int dlt = qb - kb;
-          on = kb == 0 || sv[kb] || offset_on(dlt) || offset_on(dlt - 1);
+          on = kb == 0 || sv[kb] || slash_hit(kb);
         } else {
           on = kb == 0 || kb == qb || st.all;
           if (!st.all) {
@@ -515,7 +542,7 @@ __global__ void __launch_bounds__(256) build_tiles_kernel(crisp_params p, const 
     if (mrow) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
-        if (base + lane * 4 + i < nb) mrow[base + lane * 4 + i] = f[i];
+        if (base + lane * 4 + i < nbs) mrow[base + lane * 4 + i] = f[i];
     }
     int c = int(f[0]) + int(f[1]) + int(f[2]) + int(f[3]);
     int pre = c;
@@ -531,11 +558,11 @@ __global__ void __launch_bounds__(256) build_tiles_kernel(crisp_params p, const 
     count += __shfl_sync(0xffffffffu, pre, 31);
     if (base + 128 > qb) {
       // the rest of the row lies above the diagonal: mask zeros only
-      for (int b2 = base + 128 + lane; mrow && b2 < nb; b2 += 32) mrow[b2] = 0;
+      for (int b2 = base + 128 + lane; mrow && b2 < nbs; b2 += 32) mrow[b2] = 0;
       break;
     }
   }
-  if (lane == 0) tile_cnt[size_t(bh) * nb + qb] = count;
+  if (lane == 0) tile_cnt[size_t(bh) * nbs + qb] = count;
 }
 
 // ---------------------------------------------------------------------------
@@ -545,7 +572,7 @@ cudaError_t run_select(const crisp_params& p, const void* q, const void* k, cons
                        const float* p_v, const float* p_s, void* ws, uint8_t* mask,
                        int32_t* tile_idx, int32_t* tile_cnt, cudaStream_t st) {
   const Workspace W = make_workspace(p);
-  const int nb = p.seqlen / p.block;
+  const int nb = n_blocks(p);
   const int BH = p.batch * p.h_q;
   cudaError_t e;
   // (1) VS selection per direction.

@@ -28,11 +28,23 @@
  *    completion counters its kernels keep right after it); a caller who runs
  *    crisp_select or crisp_sparse_prefill alone on a new workspace zeroes
  *    those 8 bytes.
- *  - Block geometry: N_b = seqlen / block. seqlen must be a multiple of 128
- *    and of block; block is 64 or 128; head_dim is 64 or 128;
+ *  - Block geometry: N_b = ceil(n / block) for a sequence of n tokens
+ *    (CRISP paper, Section 4.3); the last block may be partial. block is 64
+ *    or 128; head_dim is 64 or 128; with N_b = ceil(seqlen / block),
  *    3 <= N_b <= 8192 and ceil(N_b / 64) <= block; batch * h_q <= 65535 and
  *    batch * h_q * seqlen < 2^31 (rows of q addressed by 32-bit tile
  *    coordinates). Anything else returns CRISP_ERR_SHAPE.
+ *  - Variable lengths: with p->seq_lens == NULL every sequence has seqlen
+ *    tokens. Otherwise seq_lens is a DEVICE array of batch int32 lengths
+ *    and sequence b occupies the first seq_lens[b] rows of its
+ *    [seqlen][head_dim] slices; the other rows are padding that no result
+ *    depends on. Each length must satisfy 2*block < n <= seqlen (N_b >= 3);
+ *    a kernel that meets one outside clamps it into that range and records
+ *    CRISP_ERR_DEVICE. Padding rows of v must hold finite values up to the
+ *    next multiple of 128 rows (the tensor cores multiply them by exact
+ *    zeros; zeros are the natural filler). Per-block outputs beyond a
+ *    sequence's own N_b are zero (p_v, p_s, tile_cnt, mask, vs_sel); rows
+ *    of o beyond its length are zero and their lse is -inf.
  *  - Return codes: CRISP_OK, or a negative crisp_status. Invalid arguments
  *    never launch a kernel.
  */
@@ -75,6 +87,7 @@ typedef struct {
   int32_t router;      /* crisp_router */
   int32_t vs_rule;     /* crisp_vs_rule */
   float sm_scale;      /* softmax scale; 0 selects 1/sqrt(head_dim) */
+  const int32_t* seq_lens; /* device [batch] sequence lengths, or NULL (all = seqlen) */
 } crisp_params;
 
 /* Library version (major*10000 + minor*100 + patch). */
@@ -114,7 +127,10 @@ int crisp_route(const crisp_params* p, const void* q, const void* k, void* ws, s
  * (vs_rule GAMMA: smallest prefix of the descending scores reaching gamma,
  * clipped the same way); the union with vertical block 0 and slash block
  * N_b-1 marks tile (qb, kb <= qb) iff kb is a selected vertical block or
- * qb-kb or qb-kb-1 is a selected slash offset (offset = N_b-1-slash id).
+ * the tile holds a causal (t, j) pair whose slash index j + n-1-t falls in a
+ * selected slash block: for n a multiple of block, iff qb-kb or qb-kb-1 is
+ * a selected slash offset (offset = N_b-1-slash id); for a partial last
+ * block a slash block can meet three tile diagonals.
  * PE heads: Algorithm 4 — block-mean pooling of Q and K, causal block
  * softmax, entries divided by N_b, smallest descending prefix reaching
  * gamma (ties to the lower flat id qb*N_b+kb), plus tiles (qb,qb), (qb,0).

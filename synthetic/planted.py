@@ -83,6 +83,10 @@ WORKLOADS: Dict[str, Workload] = {
     "llama_32k": Workload("llama_32k", 1, 32, 8, 128, 32768, 128),
     "qwen_131k": Workload("qwen_131k", 1, 28, 4, 128, 131072, 128, sink_logit_range=(1.0, 6.0)),
     "llama_512k": Workload("llama_512k", 1, 32, 8, 128, 524288, 128),
+    # four prompts of different lengths (none a multiple of the block but the
+    # first) in one padded batch
+    "llama_varlen_131k": Workload("llama_varlen_131k", 4, 32, 8, 128, 131072, 128,
+                                  lengths=(131072, 98304 + 37, 65536 + 1, 32768 + 123)),
 }
 
 

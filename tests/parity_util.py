@@ -24,8 +24,9 @@ def run_gpu(w, q, k, v, router="cstruct", vs_rule="alpha", alpha=1.0, gamma=0.95
     """Runs route -> select -> sparse prefill through the C ABI; returns CPU copies."""
     import dynamic_block_sparse_qk_b200 as C
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    lens = None if w.lengths is None else torch.tensor(list(w.lengths), dtype=torch.int32, device=qd.device)
     p = C.params_for(qd, kd, block=w.block, alpha=alpha, gamma=gamma, router=router,
-                     vs_rule=vs_rule, tau_jsd=tau_jsd)
+                     vs_rule=vs_rule, tau_jsd=tau_jsd, seq_lens=lens)
     ws = C.alloc_workspace(p, qd.device)
     pattern, score, p_v, p_s = C.crisp_route(p, qd, kd, ws)
     nb = p.n_blocks
@@ -38,7 +39,7 @@ def run_gpu(w, q, k, v, router="cstruct", vs_rule="alpha", alpha=1.0, gamma=0.95
     out = {key: val.cpu() for key, val in out.items()}
     out["status"] = status
     out["params"] = p
-    del qd, kd, vd, ws
+    del qd, kd, vd, ws, lens
     torch.cuda.empty_cache()
     return out
 
@@ -112,13 +113,16 @@ def pe_exempt(a_bar: np.ndarray, gamma: float) -> np.ndarray:
 def compare_head(gpu, b, h, q_head, k_head, v_head, w, oprm, qblocks=None, score_tol=2e-5):
     """Compares one query head; returns a report dict (asserts on hard failures)."""
     bh = b * w.h_q + h
-    nb = w.n_blocks
+    n = q_head.shape[0]                        # this sequence's length
+    nb = O.n_blocks(n, w.block)                # its blocks; GPU arrays are w.n_blocks wide
     rep = {"head": (b, h), "exempt_route": False, "exempt_blocks": 0}
     orc = O.head_route_and_select(q_head, k_head, oprm)
     gp = int(gpu["pattern"][bh])
-    # (1) block scores
-    np.testing.assert_allclose(gpu["p_v"][bh].double().numpy(), orc["p_v"], rtol=score_tol, atol=1e-9)
-    np.testing.assert_allclose(gpu["p_s"][bh].double().numpy(), orc["p_s"], rtol=score_tol, atol=1e-9)
+    # (1) block scores (zero past the sequence's own blocks)
+    for key in ("p_v", "p_s"):
+        row = gpu[key][bh].double().numpy()
+        np.testing.assert_allclose(row[:nb], orc[key], rtol=score_tol, atol=1e-9)
+        assert not row[nb:].any(), key
     # (2) route
     tau = oprm.tau_jsd if oprm.router == "jsd" else oprm.tau_proxy
     np.testing.assert_allclose(float(gpu["score"][bh]), orc["score"], rtol=score_tol, atol=1e-7)
@@ -129,10 +133,14 @@ def compare_head(gpu, b, h, q_head, k_head, v_head, w, oprm, qblocks=None, score
     else:
         assert gp == orc["routed"], (b, h, gp, orc["routed"], orc["score"])
     rep["pattern"] = gp
-    gmask = gpu["mask"][bh].numpy().astype(bool)
+    full_mask = gpu["mask"][bh].numpy().astype(bool)
+    assert not full_mask[nb:].any() and not full_mask[:, nb:].any()
+    gmask = full_mask[:nb, :nb]
     # (3) selection
     if gp == O.VS:
-        sel = gpu["vs_sel"][bh].numpy().astype(bool)
+        sel_full = gpu["vs_sel"][bh].numpy().astype(bool)
+        assert not sel_full[:, nb:].any()
+        sel = sel_full[:, :nb]
         for d, (key, pd) in enumerate((("s_v", orc["p_v"]), ("s_s", orc["p_s"]))):
             want = np.zeros(nb, dtype=bool)
             want[orc[key]] = True
@@ -142,7 +150,7 @@ def compare_head(gpu, b, h, q_head, k_head, v_head, w, oprm, qblocks=None, score
             rep["exempt_blocks"] += int(ex.sum())
         s_v = np.nonzero(sel[0])[0]
         s_s = np.nonzero(sel[1])[0]
-        np.testing.assert_array_equal(gmask, O.vs_tile_mask(s_v, s_s, nb))
+        np.testing.assert_array_equal(gmask, O.vs_tile_mask(s_v, s_s, nb, n, w.block))
     else:
         ex = pe_exempt(orc["a_bar"], oprm.gamma)
         want = orc["mask"]
@@ -153,7 +161,9 @@ def compare_head(gpu, b, h, q_head, k_head, v_head, w, oprm, qblocks=None, score
         assert not np.triu(gmask, 1).any()
         rep["exempt_blocks"] += int(ex.sum())
     # (4) tile lists = ascending nonzeros of the mask row
-    cnt = gpu["tile_cnt"][bh].numpy()
+    cnt_full = gpu["tile_cnt"][bh].numpy()
+    assert not cnt_full[nb:].any()
+    cnt = cnt_full[:nb]
     np.testing.assert_array_equal(cnt, gmask.sum(axis=1))
     tidx = gpu["tile_idx"][bh].numpy()
     for qb in range(nb):
@@ -162,8 +172,11 @@ def compare_head(gpu, b, h, q_head, k_head, v_head, w, oprm, qblocks=None, score
     # (5) attention on the GPU's own mask
     o_ref, lse_ref, rows = O.masked_attention_rows(q_head, k_head, v_head, gmask, w.block,
                                                    oprm.scale(q_head.shape[1]), qblocks)
-    o_gpu = gpu["o"][b, h].float().numpy()[rows]
-    lse_gpu = gpu["lse"][b, h].numpy()[rows]
+    o_all = gpu["o"][b, h].float().numpy()
+    lse_all = gpu["lse"][b, h].numpy()
+    assert not o_all[n:].any() and np.all(lse_all[n:] == -np.inf)     # padding rows
+    o_gpu = o_all[rows]
+    lse_gpu = lse_all[rows]
     err = np.abs(o_gpu - o_ref)
     rep["attn_max_abs"] = float(err.max())
     rep["attn_mean_abs"] = float(err.mean())
@@ -185,9 +198,10 @@ def compare_all(w, q, k, v, gpu, oprm, qblocks_fn=None, heads=None):
     reports = []
     for b in range(w.batch):
         for h in (range(w.h_q) if heads is None else heads):
-            qh = O.bf16_to_f64(q[b, h])
-            kh = O.bf16_to_f64(k[b, h // g])
-            vh = O.bf16_to_f64(v[b, h // g])
+            n = w.length(b)
+            qh = O.bf16_to_f64(q[b, h, :n])
+            kh = O.bf16_to_f64(k[b, h // g, :n])
+            vh = O.bf16_to_f64(v[b, h // g, :n])
             qbs = None if qblocks_fn is None else qblocks_fn(b, h)
             reports.append(compare_head(gpu, b, h, qh, kh, vh, w, oprm, qbs))
     return reports

@@ -84,6 +84,75 @@ def test_edge_shapes(kw):
     _check(Workload(**base))
 
 
+# ---- sequences whose length is not a multiple of the block (N_b = ceil(n / B)),
+# and batches of different lengths stored with padding rows
+@pytest.mark.parametrize("kw", [
+    dict(seqlen=2048 + 37, block=64, head_dim=64, h_q=2, h_kv=1),          # tiny shape, 37-row last block
+    dict(seqlen=5 * 128 + 1, block=128, head_dim=128, h_q=4, h_kv=2),      # one-token last block
+    dict(seqlen=3 * 128 - 1, block=128, head_dim=128, h_q=2, h_kv=1),      # N_b = 3, 127-row last block
+    dict(seqlen=1000, block=64, head_dim=64, h_q=4, h_kv=1),               # GQA g = 4, 40-row last block
+    dict(seqlen=4096 + 77, block=128, head_dim=64, h_q=2, h_kv=2),         # d = 64 at B = 128
+])
+def test_ragged_single_sequence(kw):
+    base = dict(name="ragged", batch=1, n_vertical=2, diffuse_frac=0.5, sink_logit=8.0)
+    base.update(kw)
+    _check(Workload(**base))
+
+
+@pytest.mark.parametrize("router,vs_rule", [("jsd", "alpha"), ("cstruct", "gamma"), ("cstruct", "alpha_median")])
+def test_ragged_router_and_rules(router, vs_rule):
+    w = Workload("ragged_r", 1, 4, 2, 128, 2048 + 93, 128, n_vertical=2, diffuse_frac=0.5, sink_logit=8.0)
+    _check(w, router=router, vs_rule=vs_rule)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(batch=3, seqlen=2048, block=128, head_dim=128, h_q=4, h_kv=2, lengths=(2048, 1500, 257)),
+    dict(batch=2, seqlen=1536 + 64, block=64, head_dim=64, h_q=2, h_kv=1, lengths=(777, 1600)),
+    dict(batch=2, seqlen=4096, block=128, head_dim=128, h_q=8, h_kv=2, lengths=(4096 - 1, 2 * 128 + 1)),
+])
+def test_variable_length_batch(kw):
+    base = dict(name="varlen", n_vertical=2, diffuse_frac=0.5, sink_logit=8.0)
+    base.update(kw)
+    _check(Workload(**base))
+
+
+def test_variable_length_dense_equals_oracle():
+    w = Workload("varlen_dense", 2, 2, 1, 128, 1536, 128, lengths=(1536 - 100, 700))
+    q, k, v, _ = make_qkv(w)
+    import dynamic_block_sparse_qk_b200 as C
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    lens = torch.tensor(w.lengths, dtype=torch.int32, device="cuda")
+    p = C.params_for(qd, kd, block=128, seq_lens=lens)
+    ws = C.alloc_workspace(p)
+    o, lse = C.crisp_dense_prefill(p, qd, kd, vd, ws)
+    assert C.crisp_get_device_status(ws) == 0
+    o, lse = o.float().cpu().numpy(), lse.cpu().numpy()
+    for b, n in enumerate(w.lengths):
+        nb = O.n_blocks(n, 128)
+        full = np.tril(np.ones((nb, nb), dtype=bool))
+        for h in range(2):
+            ref, lref, rows = O.masked_attention_rows(O.bf16_to_f64(q[b, h, :n]), O.bf16_to_f64(k[b, 0, :n]),
+                                                      O.bf16_to_f64(v[b, 0, :n]), full, 128, 128 ** -0.5)
+            err = np.abs(o[b, h, :n] - ref)
+            assert err.max() <= 2e-2 and err.mean() <= 2e-3
+            np.testing.assert_allclose(lse[b, h, :n], lref, atol=2e-3)
+            assert not o[b, h, n:].any() and np.all(lse[b, h, n:] == -np.inf)
+
+
+def test_length_out_of_range_is_reported_and_clamped():
+    w = Workload("badlen", 2, 2, 1, 64, 1024, 64, lengths=(1024, 1024))
+    q, k, v, _ = make_qkv(w)
+    import dynamic_block_sparse_qk_b200 as C
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    lens = torch.tensor([1024, 100], dtype=torch.int32, device="cuda")   # 100 <= 2 * block
+    p = C.params_for(qd, kd, block=64, seq_lens=lens)
+    ws = C.alloc_workspace(p)
+    pattern, score, pv, ps = C.crisp_route(p, qd, kd, ws)
+    C.crisp_select(p, qd, kd, pattern, pv, ps, ws)
+    assert C.crisp_get_device_status(ws) == -6
+    assert C.crisp_get_device_status(ws) == 0
+
+
 def test_kmin_above_nb():
     w = Workload("kmin", 1, 2, 1, 64, 512, 64, diffuse_heads=(1,), n_vertical=0, sink_logit=8.0)
     q, k, v, _ = make_qkv(w)
@@ -159,6 +228,13 @@ def test_llama_32k_median_floor():
     w = WORKLOADS["llama_32k"]
     reps = _check(w, vs_rule="alpha_median", qblocks_fn=lambda b, h: PU.sample_qblocks(w.n_blocks, 2, 1500 + h))
     assert sum(r["pattern"] == O.VS for r in reps) == 24
+
+
+def test_variable_length_llama_32k():
+    w = WORKLOADS["llama_32k"].with_(name="llama_32k_varlen", batch=2, lengths=(32768 - 5, 20000 + 37))
+    reps = _check(w, qblocks_fn=lambda b, h: PU.sample_qblocks(O.n_blocks(w.length(b), 128), 2, 4000 + h),
+                  heads=range(0, 32, 3))
+    assert {r["pattern"] for r in reps} == {O.VS, O.PE}
 
 
 @pytest.mark.slow
