@@ -54,6 +54,8 @@ class CrispParams:
     router: str = "cstruct"   # "cstruct" (Eq. 2) or "jsd" (Appendix A, Algorithm 5)
     vs_rule: str = "alpha"    # "alpha" (Algorithm 3), "alpha_median" (Algorithm 3 with the
                               # median floor of Appendix H) or "gamma" (Appendix A, Algorithm 6)
+    granularity: str = "tile" # VS mask of Eq. 1: "tile" (selected blocks as whole tiles) or
+                              # "token" (slash blocks as diagonal bands inside the tiles)
     sm_scale: float = 0.0     # 0 -> 1/sqrt(d)
 
     def scale(self, d: int) -> float:
@@ -391,9 +393,16 @@ def pe_tile_mask(selected_flat: np.ndarray, nb: int) -> np.ndarray:
 
 
 def masked_attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, tile_mask: np.ndarray,
-                          block: int, scale: float, qblocks: Optional[Sequence[int]] = None):
+                          block: int, scale: float, qblocks: Optional[Sequence[int]] = None,
+                          vs_tokens: Optional[tuple] = None):
     """Eq. 1: O = Softmax(Q K^T * scale + M_S) V with M_S from whole tiles
     and the causal mask; float64 throughout.
+
+    With vs_tokens = (S_v, S_s) the mask of a VS head is taken at token
+    granularity inside those tiles: query t sees key j iff block(j) is a
+    selected vertical block (or block 0) or the slash index j + n - 1 - t lies
+    in a selected slash block (or block N_b - 1) — Eq. 1's M_S with
+    j in S_t read token by token.
 
     Returns (O [len(rows), d], lse [len(rows)], rows) for the listed query
     blocks (all when None). lse is the natural-log sum of exp of the logits.
@@ -401,6 +410,13 @@ def masked_attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, tile_mask
     n, d = q.shape
     nb = n_blocks(n, block)
     qbs = list(range(nb)) if qblocks is None else list(qblocks)
+    if vs_tokens is not None:
+        col_on = np.zeros(nb, dtype=bool)
+        col_on[np.asarray(vs_tokens[0], dtype=np.int64)] = True
+        col_on[0] = True
+        slash_on = np.zeros(nb, dtype=bool)
+        slash_on[np.asarray(vs_tokens[1], dtype=np.int64)] = True
+        slash_on[nb - 1] = True
     outs, lses, rows = [], [], []
     for qb in qbs:
         kbs = np.nonzero(tile_mask[qb, : qb + 1])[0]
@@ -408,7 +424,11 @@ def masked_attention_rows(q: np.ndarray, k: np.ndarray, v: np.ndarray, tile_mask
         keys = keys[keys < n]
         t = np.arange(qb * block, min(qb * block + block, n))
         z = (q[t] @ k[keys].T) * scale
-        z = np.where(keys[None, :] <= t[:, None], z, -np.inf)
+        seen = keys[None, :] <= t[:, None]
+        if vs_tokens is not None:
+            sl = (keys[None, :] + n - 1 - t[:, None]) // block
+            seen &= col_on[keys // block][None, :] | slash_on[np.clip(sl, 0, nb - 1)]
+        z = np.where(seen, z, -np.inf)
         m = z.max(axis=1, keepdims=True)
         e = np.exp(z - m)
         s = e.sum(axis=1, keepdims=True)
@@ -462,6 +482,8 @@ def head_route_and_select(q_head: np.ndarray, k_head: np.ndarray, prm: CrispPara
             raise ValueError(f"unknown vs_rule {prm.vs_rule!r}")
         out["s_v"], out["s_s"] = s_v, s_s
         out["mask"] = vs_tile_mask(s_v, s_s, nb, n, B)
+        if prm.granularity == "token":
+            out["vs_tokens"] = (s_v, s_s)
     else:
         a_bar = pe_estimate(pe_pool(q_head, B), pe_pool(k_head, B), scale)
         sel = pe_index(a_bar, prm.gamma)
@@ -498,5 +520,6 @@ def crisp_prefill(q, k, v, prm: CrispParams, qblocks: Optional[Sequence[int]] = 
             hr = head_route_and_select(qh, kh, prm, force_pattern=fp)
             res["heads"][(b, h)] = hr
             mask = hr["mask"] if masks is None else masks[(b, h)]
-            res["attn"][(b, h)] = masked_attention_rows(qh, kh, vh, mask, prm.block, scale, qblocks)
+            res["attn"][(b, h)] = masked_attention_rows(qh, kh, vh, mask, prm.block, scale, qblocks,
+                                                        hr.get("vs_tokens"))
     return res

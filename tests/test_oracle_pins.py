@@ -491,6 +491,41 @@ def test_ragged_full_mask_equals_dense_causal_softmax():
         np.testing.assert_allclose(lse, want_lse, atol=1e-13)
 
 
+def test_token_granular_vs_mask_bruteforce():
+    # Eq. 1 with S_t read token by token: vertical blocks whole, slash blocks as
+    # diagonal bands; aligned and ragged n
+    rng = _rng(25)
+    B = 8
+    for n in (40, 43, 57):
+        nb = -(-n // B)
+        q, k, v = rng.standard_normal((3, n, 4))
+        s_v = rng.choice(nb, size=2, replace=False)
+        s_s = rng.choice(nb, size=2, replace=False)
+        cols = set(int(x) for x in s_v) | {0}
+        slash = set(int(x) for x in s_s) | {nb - 1}
+        tiles = O.vs_tile_mask(s_v, s_s, nb, n, B)
+        o, lse, _ = O.masked_attention_rows(q, k, v, tiles, B, 0.5, vs_tokens=(s_v, s_s))
+        allowed = lambda t, j: j <= t and (j // B in cols or (j + n - 1 - t) // B in slash)
+        want_o, want_lse = _attention_bruteforce(q.tolist(), k.tolist(), v.tolist(), allowed, 0.5)
+        np.testing.assert_allclose(o, want_o, atol=1e-13)
+        np.testing.assert_allclose(lse, want_lse, atol=1e-13)
+        # whole tiles see a superset of keys: the token-level lse is never larger
+        _, lse_tile, _ = O.masked_attention_rows(q, k, v, tiles, B, 0.5)
+        assert np.all(lse <= lse_tile + 1e-12)
+
+
+def test_token_granular_equals_tiles_when_every_slash_block_is_kept():
+    rng = _rng(26)
+    B, n = 8, 45
+    nb = -(-n // B)
+    q, k, v = rng.standard_normal((3, n, 4))
+    every = np.arange(nb)
+    tiles = O.vs_tile_mask([3], every, nb, n, B)
+    a = O.masked_attention_rows(q, k, v, tiles, B, 0.7, vs_tokens=([3], every))
+    b = O.masked_attention_rows(q, k, v, tiles, B, 0.7)
+    np.testing.assert_allclose(a[0], b[0], atol=1e-14)
+
+
 def test_prefill_lengths_ignore_padding():
     rng = _rng(24)
     B, N = 8, 48
