@@ -141,7 +141,7 @@ def run_ours(args, rank, world, local_rank):
     q, k, v, meta = make_qkv(w, device=str(dev))
     lens = None if w.lengths is None else torch.tensor(list(w.lengths), dtype=torch.int32, device=dev)
     p = C.params_for(q, k, block=w.block, alpha=args.alpha, gamma=args.gamma, router=args.router,
-                     vs_rule=args.vs_rule, seq_lens=lens)
+                     vs_rule=args.vs_rule, seq_lens=lens, granularity=args.granularity)
     ws = C.alloc_workspace(p, dev)
     bh, nb = p.batch * p.h_q, p.n_blocks
     pattern = torch.empty(bh, dtype=torch.int32, device=dev)
@@ -258,7 +258,8 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": w.name, "batch": w.batch, "h_q": w.h_q, "h_kv": w.h_kv,
                    "head_dim": w.head_dim, "seq_len": w.seqlen, "block": w.block,
                    "diffuse_frac": w.diffuse_frac, "alpha": args.alpha, "gamma": args.gamma,
-                   "router": args.router, "vs_rule": args.vs_rule, "parallelism": f"replicas{world}",
+                   "router": args.router, "vs_rule": args.vs_rule, "granularity": args.granularity,
+                   "parallelism": f"replicas{world}",
                    **({"lengths": list(w.lengths)} if w.lengths is not None else {}),
                    "l2": "flushed between steps" if flush is not None else
                          f"inputs ({in_bytes / 2**30:.1f} GiB) larger than L2"},
@@ -399,7 +400,7 @@ def oracle_sample(w, args, inp, budget_s: float):
 
     g = w.h_q // w.h_kv
     prm = O.CrispParams(block=w.block, alpha=args.alpha, gamma=args.gamma, router=args.router,
-                        vs_rule=args.vs_rule)
+                        vs_rule=args.vs_rule, granularity=args.granularity)
     nb = w.n_blocks
     sel_ms, tiles, attn_ms_per_tile = {}, {}, []
     t_start = time.perf_counter()
@@ -416,7 +417,8 @@ def oracle_sample(w, args, inp, budget_s: float):
             if time.perf_counter() - t_start > budget_s:
                 break
             t0 = time.perf_counter()
-            O.masked_attention_rows(qh, kh, vh, r["mask"], w.block, prm.scale(w.head_dim), [qb])
+            O.masked_attention_rows(qh, kh, vh, r["mask"], w.block, prm.scale(w.head_dim), [qb],
+                                    r.get("vs_tokens"))
             attn_ms_per_tile.append((time.perf_counter() - t0) * 1e3 / max(int(r["mask"][qb].sum()), 1))
     n_pe = inp["n_diffuse"]
     n_vs = w.h_q - n_pe
@@ -469,6 +471,8 @@ def main():
     ap.add_argument("--gamma", type=float, default=0.95)
     ap.add_argument("--router", default="cstruct")
     ap.add_argument("--vs-rule", default="alpha", choices=["alpha", "alpha_median", "gamma"])
+    ap.add_argument("--granularity", default="tile", choices=["tile", "token"],
+                    help="VS mask: selected blocks as whole tiles, or slash blocks as diagonal bands")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -21,6 +21,8 @@ STATUS_NAMES = {0: "ok", -1: "invalid argument", -2: "unsupported shape", -3: "w
                 -4: "CUDA error", -5: "device wait timed out", -6: "device index out of range"}
 ROUTER = {"cstruct": 0, "jsd": 1}
 VS_RULE = {"alpha": 0, "gamma": 1, "alpha_median": 2}
+GRANULARITY = {"tile": 0, "token": 1}
+TILE_ID_MASK, TILE_WHOLE, TILE_SLASH_SHIFT = 0xFFFFFF, 1 << 24, 25
 PATTERN_VS, PATTERN_PE = 0, 1
 
 EXPORTED = ("crisp_version", "crisp_status_string", "crisp_check_params", "crisp_workspace_size",
@@ -43,7 +45,7 @@ class CrispParams(ctypes.Structure):
                 ("alpha", ctypes.c_float), ("gamma", ctypes.c_float), ("tau_proxy", ctypes.c_float),
                 ("tau_jsd", ctypes.c_float), ("k_min_blocks", ctypes.c_int32),
                 ("router", ctypes.c_int32), ("vs_rule", ctypes.c_int32), ("sm_scale", ctypes.c_float),
-                ("seq_lens", ctypes.c_void_p)]
+                ("vs_granularity", ctypes.c_int32), ("seq_lens", ctypes.c_void_p)]
 
     @property
     def n_blocks(self) -> int:
@@ -53,7 +55,7 @@ class CrispParams(ctypes.Structure):
 
 def make_params(batch, h_q, h_kv, seqlen, head_dim, block=128, alpha=1.0, gamma=0.95,
                 tau_proxy=0.2, tau_jsd=0.1, k_min_blocks=8, router="cstruct", vs_rule="alpha",
-                sm_scale=0.0, seq_lens: Optional[torch.Tensor] = None) -> CrispParams:
+                sm_scale=0.0, seq_lens: Optional[torch.Tensor] = None, granularity="tile") -> CrispParams:
     """seq_lens: optional CUDA int32 tensor [batch] of sequence lengths. The
     params keep only its device address: keep the tensor alive while they are
     in use."""
@@ -64,6 +66,7 @@ def make_params(batch, h_q, h_kv, seqlen, head_dim, block=128, alpha=1.0, gamma=
     p = CrispParams(batch, h_q, h_kv, seqlen, head_dim, block, alpha, gamma, tau_proxy, tau_jsd,
                     k_min_blocks, ROUTER[router] if isinstance(router, str) else int(router),
                     VS_RULE[vs_rule] if isinstance(vs_rule, str) else int(vs_rule), sm_scale,
+                    GRANULARITY[granularity] if isinstance(granularity, str) else int(granularity),
                     None if seq_lens is None else seq_lens.data_ptr())
     return p
 

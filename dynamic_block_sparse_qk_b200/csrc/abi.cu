@@ -32,6 +32,8 @@ int check_params(const crisp_params* p) {
   if (p->vs_rule != CRISP_VS_ALPHA && p->vs_rule != CRISP_VS_GAMMA && p->vs_rule != CRISP_VS_ALPHA_MEDIAN)
     return CRISP_ERR_ARG;
   if (!(p->sm_scale >= 0.f) || !isfinite(p->sm_scale)) return CRISP_ERR_ARG;
+  if (p->vs_granularity != CRISP_GRAN_TILE && p->vs_granularity != CRISP_GRAN_TOKEN) return CRISP_ERR_ARG;
+  if (p->vs_granularity == CRISP_GRAN_TOKEN && p->block != 128) return CRISP_ERR_SHAPE;
   return CRISP_OK;
 }
 
@@ -49,7 +51,7 @@ int to_status(cudaError_t e) { return e == cudaSuccess ? CRISP_OK : CRISP_ERR_CU
 
 extern "C" {
 
-int crisp_version(void) { return 10100; }
+int crisp_version(void) { return 10200; }
 
 const char* crisp_status_string(int s) {
   switch (s) {

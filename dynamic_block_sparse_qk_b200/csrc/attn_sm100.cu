@@ -69,21 +69,26 @@ struct Cfg {
 
 // Walks the 128-key tiles a query tile needs, ascending, with membership bits:
 // bit (i * kpu + ks) says query block qb0+i attends key block kt*kpu+ks.
+// Bits 8..11 carry the token-granularity flags of the tile (bit 8: whole
+// tile; bits 9..11: slash blocks N_b-1-delta+e selected, e = -1, 0, +1); a
+// dense walk, tile-granularity lists and 64-wide blocks mark every tile whole.
+constexpr uint32_t kStepWhole = 1u << 8;
 struct StepIter {
   const int32_t* lst[2];
   int cnt[2], pos[2];
   int nsub, kpu, qb0, dense_last, next_kt;
   int ahead;        // single list: the next entry, already loaded (-2: none)
   int32_t* status;
-  bool report;
+  bool report, token;
 
   __device__ void init(const int32_t* tile_idx, const int32_t* tile_cnt, int bh, int nb, int block,
-                       int qt, int32_t* st, bool rep) {
+                       int qt, int32_t* st, bool rep, bool tok) {
     nsub = BM / block;
     kpu = BN / block;
     qb0 = qt * nsub;
     status = st;
     report = rep;
+    token = tok && nsub == 1;
     next_kt = 0;
     dense_last = tile_idx ? -1 : qt;
     for (int i = 0; i < 2; ++i) { lst[i] = nullptr; cnt[i] = 0; pos[i] = 0; }
@@ -110,7 +115,7 @@ struct StepIter {
     if (dense_last >= 0) {
       if (next_kt > dense_last) return false;
       kt = next_kt++;
-      bits = 0;
+      bits = kStepWhole;
       for (int i = 0; i < nsub; ++i)
         for (int ks = 0; ks < kpu; ++ks)
           if (kt * kpu + ks <= qb0 + i) bits |= 1u << (i * kpu + ks);
@@ -122,9 +127,10 @@ struct StepIter {
         const int v = ahead;
         ++pos[0];
         ahead = pos[0] < cnt[0] ? lst[0][pos[0]] : -2;
-        if (v >= 0 && v <= qb0) {
-          kt = v / kpu;
-          bits = 1u << (v % kpu);
+        const int id = token ? (v & kTileIdMask) : v;
+        if (v >= 0 && id <= qb0) {
+          kt = id / kpu;
+          bits = (1u << (id % kpu)) | (token ? ((uint32_t(v) >> 24) & 15u) << 8 : kStepWhole);
           return true;
         }
         if (report) report_error(status, CRISP_ERR_DEVICE, v);
@@ -144,7 +150,7 @@ struct StepIter {
       if (pos[i] < cnt[i]) best = min(best, lst[i][pos[i]] / kpu);
     }
     if (best == INT_MAX) return false;
-    bits = 0;
+    bits = kStepWhole;
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       if (i >= nsub) break;
@@ -165,7 +171,7 @@ struct StepIter {
   }
 };
 
-template <int D, int BLK>
+template <int D, int BLK, bool TOKEN>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                    const __grid_constant__ CUtensorMap tmv, const int32_t* __restrict__ tile_idx,
@@ -186,6 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Workspace W = make_workspace(p);
   int32_t* status = ws_ptr<int32_t>(ws, W.status);
   const int N = p.seqlen, nb = n_blocks(p), NT = (N + BM - 1) / BM;
+  constexpr bool token = TOKEN;   // token-granular slash bands (block 128 lists only)
   // Work order: KV-head major (the CTAs running at the same time read the same
   // K/V stream, which then stays in L2), longest query tiles first inside.
   const int g = p.h_q / p.h_kv;
@@ -251,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ring = is_k ? sRing : sVRing;
       const int bfull = is_k ? C::B_KFULL : C::B_VFULL, bempty = is_k ? C::B_KEMPTY : C::B_VEMPTY;
       StepIter it;
-      it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, is_k);
+      it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, is_k, token);
       if (is_k) {
         mbar_arrive_expect_tx(BAR(C::B_Q), C::Q_BYTES);
         for (int box = 0; box < D / 64; ++box)
@@ -280,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ UMMA issuer: S_j = Q K_j^T
     if (lane == 0) {
       StepIter it;
-      it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, false);
+      it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, false, token);
       constexpr uint32_t idq = idesc_bf16(BM, BN, 0);
       bool ok = mbar_wait(BAR(C::B_Q), 0, abort_flag, status, 4);
       int j = 0, kt;
@@ -311,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ UMMA issuer: O += P V
     if (lane == 0) {
       StepIter it;
-      it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, false);
+      it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, false, token);
       constexpr uint32_t idp = idesc_bf16(BM, D, 1);
       bool ok = true;
       int j = 0, kt;
@@ -353,7 +360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qsub = r / BLK;
     const float sl2 = (p.sm_scale > 0.f ? p.sm_scale : rsqrtf(float(D))) * kLog2e;
     StepIter it;
-    it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, false);
+    it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, false, token);
     float m_use = -INFINITY, l = 0.f;
     int j = grp, u = 0, kt, kt_next;
     uint32_t bits, bits_next;
@@ -386,6 +393,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(rb & 2u)) hi = min(hi, BLK - 1);
       } else if (!rb) {
         hi = -1;
+      }
+      if (TOKEN && !(bits & kStepWhole)) {
+        // Token granularity (block 128): only the diagonal bands of the
+        // selected slash blocks N_b-1-delta+e, e = -1, 0, +1; for this row the
+        // band of e covers columns [r - s + e B, r - s + e B + B - 1],
+        // s = (len - 1) mod B. Inside the tile the bands e = -1 and e = +1
+        // exclude each other (the first needs r > s, the second r < s), so
+        // the selected bands always leave one window per row.
+        const uint32_t f = (bits >> 9) & 7u;
+        const int s_res = (len - 1) & (BLK - 1);
+        const int a = r - s_res - BN;
+        int wlo = 1, whi = 0;
+        if (f == 5u) {
+          wlo = r > s_res ? a : a + 2 * BN;
+          whi = wlo + BN - 1;
+        } else if (f) {
+          wlo = a + (__ffs(f) - 1) * BN;
+          whi = a + (32 - __clz(f)) * BN - 1;
+        }
+        lo = max(lo, wlo);
+        hi = min(hi, whi);
       }
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
       if (lo == 0 && hi == BN - 1) {
@@ -530,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ----------------------------------------------------------------------------- host
-template <int D, int BLK>
+template <int D, int BLK, bool TOKEN>
 cudaError_t launch_tc(const crisp_params& p, const void* q, const void* k, const void* v,
                       const int32_t* tile_idx, const int32_t* tile_cnt, void* o, float* lse, void* ws,
                       cudaStream_t st) {
@@ -539,7 +567,7 @@ cudaError_t launch_tc(const crisp_params& p, const void* q, const void* k, const
   if (!make_tmap(&mq, q, uint64_t(p.batch) * p.h_q * N, D) || !make_tmap(&mk, k, uint64_t(p.batch) * p.h_kv * N, D) ||
       !make_tmap(&mv, v, uint64_t(p.batch) * p.h_kv * N, D))
     return cudaErrorInvalidValue;
-  auto kern = attn_tc_kernel<D, BLK>;
+  auto kern = attn_tc_kernel<D, BLK, TOKEN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<D>::SMEM);
   if (e != cudaSuccess) return e;
   const unsigned grid = unsigned(p.batch) * p.h_q * ((p.seqlen + BM - 1) / BM);
@@ -553,11 +581,16 @@ cudaError_t launch_tc(const crisp_params& p, const void* q, const void* k, const
 cudaError_t run_attention(const crisp_params& p, const void* q, const void* k, const void* v,
                           const int32_t* tile_idx, const int32_t* tile_cnt, void* o, float* lse,
                           void* ws, cudaStream_t st) {
-  if (p.head_dim == 64)
-    return p.block == 64 ? launch_tc<64, 64>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st)
-                         : launch_tc<64, 128>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st);
-  return p.block == 64 ? launch_tc<128, 64>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st)
-                       : launch_tc<128, 128>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st);
+  // token-granular lists carry per-tile flags (block 128 only, checked by the ABI)
+  const bool token = tile_idx && p.vs_granularity == CRISP_GRAN_TOKEN && p.block == 128;
+  if (p.head_dim == 64) {
+    if (token) return launch_tc<64, 128, true>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st);
+    return p.block == 64 ? launch_tc<64, 64, false>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st)
+                         : launch_tc<64, 128, false>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st);
+  }
+  if (token) return launch_tc<128, 128, true>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st);
+  return p.block == 64 ? launch_tc<128, 64, false>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st)
+                       : launch_tc<128, 128, false>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st);
 }
 
 }  // namespace crisp

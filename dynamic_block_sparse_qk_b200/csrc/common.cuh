@@ -77,6 +77,12 @@ __host__ __device__ inline int proxy_chunk(const crisp_params& p) {
 
 enum HeadCounter { kCntProxy = 0, kCntHist = 1, kCntEq = 2, kCntScores = 3 };
 
+// Tile-list entries in token granularity: key-block id in the low 24 bits,
+// then flags (whole tile; slash blocks N_b-1-delta-1, N_b-1-delta, N_b-delta).
+constexpr int32_t kTileIdMask = 0xFFFFFF;
+constexpr int32_t kTileWhole = 1 << 24;
+constexpr int kTileSlashShift = 25;
+
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 __host__ __device__ inline Workspace make_workspace(const crisp_params& p) {

@@ -491,6 +491,18 @@ __global__ void __launch_bounds__(256) build_tiles_kernel(crisp_params p, const 
   const int rows_q = min(B, len - qb * B);
   const bool lo_ext = s_res - (rows_q - 1) < 0;
   auto slash_on = [&](int jb) -> bool { return jb == nb - 1 || (jb >= 0 && jb < nb && ss[jb] != 0); };
+  // List entry of an active tile: the key-block id, plus in token
+  // granularity the flags the attention kernel masks with (whole tile, or
+  // which of the three slash blocks that can meet the tile are selected).
+  const bool token = p.vs_granularity == CRISP_GRAN_TOKEN;
+  auto tile_entry = [&](int kb) -> int32_t {
+    if (!token) return kb;
+    if (!vs || kb == 0 || sv[kb]) return kb | kTileWhole;
+    int32_t v = kb;
+    for (int e = -1; e <= 1; ++e)
+      if (slash_on(nb - 1 - (qb - kb) + e)) v |= 1 << (kTileSlashShift + e + 1);
+    return v;
+  };
   auto slash_hit = [&](int kb) -> bool {
     const int dlt = qb - kb;
     const int vmax = dlt >= 1 ? B - 1 : 0;                  // key blocks before qb are full
@@ -554,7 +566,7 @@ __global__ void __launch_bounds__(256) build_tiles_kernel(crisp_params p, const 
     int pos = count + pre - c;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-      if (f[i]) idx[pos++] = base + lane * 4 + i;
+      if (f[i]) idx[pos++] = tile_entry(base + lane * 4 + i);
     count += __shfl_sync(0xffffffffu, pre, 31);
     if (base + 128 > qb) {
       // the rest of the row lies above the diagonal: mask zeros only

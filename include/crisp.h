@@ -74,6 +74,12 @@ typedef enum { CRISP_ROUTER_CSTRUCT = 0, CRISP_ROUTER_JSD = 1 } crisp_router;
  * median floor of Appendix H (Table 9). */
 typedef enum { CRISP_VS_ALPHA = 0, CRISP_VS_GAMMA = 1, CRISP_VS_ALPHA_MEDIAN = 2 } crisp_vs_rule;
 typedef enum { CRISP_PATTERN_VS = 0, CRISP_PATTERN_PE = 1 } crisp_pattern;
+/* Granularity of a VS head's mask in Eq. 1: TILE executes the selected
+ * vertical and slash blocks as whole tiles (the default); TOKEN keeps whole
+ * tiles for vertical blocks but lets a slash block admit only the key-query
+ * pairs on its diagonal band (slash index j + n-1-t in the block). TOKEN
+ * requires block 128. */
+typedef enum { CRISP_GRAN_TILE = 0, CRISP_GRAN_TOKEN = 1 } crisp_granularity;
 
 /* Problem and hyper-parameters (CRISP paper, Section 5 Setup: tau_proxy 0.2,
  * gamma 0.95 for PE, alpha 1.0, block 128, k_min 8 blocks per direction). */
@@ -87,6 +93,7 @@ typedef struct {
   int32_t router;      /* crisp_router */
   int32_t vs_rule;     /* crisp_vs_rule */
   float sm_scale;      /* softmax scale; 0 selects 1/sqrt(head_dim) */
+  int32_t vs_granularity;  /* crisp_granularity */
   const int32_t* seq_lens; /* device [batch] sequence lengths, or NULL (all = seqlen) */
 } crisp_params;
 
@@ -136,7 +143,10 @@ int crisp_route(const crisp_params* p, const void* q, const void* k, void* ws, s
  * gamma (ties to the lower flat id qb*N_b+kb), plus tiles (qb,qb), (qb,0).
  * Outputs (device): tile_cnt[b][h][N_b] (int32) and tile_idx[b][h][N_b][N_b]
  * (int32; row (b,h,qb) holds tile_cnt ascending key-block ids, the rest
- * undefined); mask[b][h][N_b][N_b] (uint8 0/1, upper triangle 0) unless
+ * undefined; with CRISP_GRAN_TOKEN each entry also carries flags above bit
+ * 24: bit 24 = whole tile (vertical block, block 0 or a PE head), bits
+ * 25..27 = slash blocks N_b-1-delta+e selected for e = -1, 0, +1, with
+ * delta = qb - kb; the key-block id is entry & 0xFFFFFF); mask[b][h][N_b][N_b] (uint8 0/1, upper triangle 0) unless
  * mask == NULL; vs_sel[b][h][2][N_b] (uint8 0/1: selected vertical, then
  * slash blocks; all 0 for PE heads) unless vs_sel == NULL.
  * pattern, p_v, p_s are crisp_route's outputs. */

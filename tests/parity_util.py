@@ -20,13 +20,14 @@ ATTN_MAX_ABS = 2e-2
 ATTN_MEAN_ABS = 2e-3
 
 
-def run_gpu(w, q, k, v, router="cstruct", vs_rule="alpha", alpha=1.0, gamma=0.95, tau_jsd=0.1):
+def run_gpu(w, q, k, v, router="cstruct", vs_rule="alpha", alpha=1.0, gamma=0.95, tau_jsd=0.1,
+            granularity="tile"):
     """Runs route -> select -> sparse prefill through the C ABI; returns CPU copies."""
     import dynamic_block_sparse_qk_b200 as C
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     lens = None if w.lengths is None else torch.tensor(list(w.lengths), dtype=torch.int32, device=qd.device)
     p = C.params_for(qd, kd, block=w.block, alpha=alpha, gamma=gamma, router=router,
-                     vs_rule=vs_rule, tau_jsd=tau_jsd, seq_lens=lens)
+                     vs_rule=vs_rule, tau_jsd=tau_jsd, seq_lens=lens, granularity=granularity)
     ws = C.alloc_workspace(p, qd.device)
     pattern, score, p_v, p_s = C.crisp_route(p, qd, kd, ws)
     nb = p.n_blocks
@@ -44,9 +45,25 @@ def run_gpu(w, q, k, v, router="cstruct", vs_rule="alpha", alpha=1.0, gamma=0.95
     return out
 
 
-def oracle_params(w, router="cstruct", vs_rule="alpha", alpha=1.0, gamma=0.95, tau_jsd=0.1):
+def oracle_params(w, router="cstruct", vs_rule="alpha", alpha=1.0, gamma=0.95, tau_jsd=0.1,
+                  granularity="tile"):
     return O.CrispParams(block=w.block, alpha=alpha, gamma=gamma, router=router, vs_rule=vs_rule,
-                         tau_jsd=tau_jsd)
+                         tau_jsd=tau_jsd, granularity=granularity)
+
+
+TILE_ID_MASK, TILE_WHOLE, TILE_SLASH_SHIFT = 0xFFFFFF, 1 << 24, 25
+
+
+def expected_token_flags(qb, kb, nb, vs, sel_v, sel_s):
+    """Flags a token-granularity list entry must carry (from the GPU's own selection)."""
+    if not vs or kb == 0 or sel_v[kb]:
+        return TILE_WHOLE
+    f = 0
+    for e in (-1, 0, 1):
+        jb = nb - 1 - (qb - kb) + e
+        if jb == nb - 1 or (0 <= jb < nb and sel_s[jb]):
+            f |= 1 << (TILE_SLASH_SHIFT + e + 1)
+    return f
 
 
 def _near(x, ref):
@@ -166,12 +183,23 @@ def compare_head(gpu, b, h, q_head, k_head, v_head, w, oprm, qblocks=None, score
     cnt = cnt_full[:nb]
     np.testing.assert_array_equal(cnt, gmask.sum(axis=1))
     tidx = gpu["tile_idx"][bh].numpy()
+    token = oprm.granularity == "token"
+    vs_tokens = None
+    if token and gp == O.VS:
+        vs_tokens = (np.nonzero(sel[0])[0], np.nonzero(sel[1])[0])
     for qb in range(nb):
-        np.testing.assert_array_equal(tidx[qb, : cnt[qb]], np.nonzero(gmask[qb])[0])
+        ids = tidx[qb, : cnt[qb]]
+        if token:
+            flags = ids & ~TILE_ID_MASK
+            ids = ids & TILE_ID_MASK
+            want = [expected_token_flags(qb, int(kb), nb, gp == O.VS, sel[0] if gp == O.VS else None,
+                                         sel[1] if gp == O.VS else None) for kb in ids]
+            np.testing.assert_array_equal(flags, want)
+        np.testing.assert_array_equal(ids, np.nonzero(gmask[qb])[0])
     rep["density"] = float(gmask.sum()) / (nb * (nb + 1) / 2)
     # (5) attention on the GPU's own mask
     o_ref, lse_ref, rows = O.masked_attention_rows(q_head, k_head, v_head, gmask, w.block,
-                                                   oprm.scale(q_head.shape[1]), qblocks)
+                                                   oprm.scale(q_head.shape[1]), qblocks, vs_tokens)
     o_all = gpu["o"][b, h].float().numpy()
     lse_all = gpu["lse"][b, h].numpy()
     assert not o_all[n:].any() and np.all(lse_all[n:] == -np.inf)     # padding rows

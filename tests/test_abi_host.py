@@ -34,7 +34,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert lib.crisp_version() == 10100
+    assert lib.crisp_version() == 10200
     assert lib.crisp_status_string(0) == b"ok"
     assert lib.crisp_status_string(-3) == b"workspace too small"
 
@@ -53,6 +53,7 @@ def _p(**kw):
     (dict(h_q=32, h_kv=0), -2),
     # batch * h_q * seqlen = 2^31 query rows: beyond 32-bit tile coordinates
     (dict(batch=64, h_q=64, h_kv=8, seqlen=2 ** 19), -2),
+    (dict(granularity=2), -1), (dict(granularity="token", block=64, seqlen=4096), -2),
 ])
 def test_check_params_rejects(lib, kw, code):
     p = _p(**kw)
@@ -64,7 +65,8 @@ def test_valid_configs_have_workspace(lib):
     for kw in (dict(), dict(batch=1, h_q=2, h_kv=1, seqlen=2048, head_dim=64, block=64),
                dict(h_q=28, h_kv=4, seqlen=131072), dict(seqlen=524288),
                dict(batch=63, h_q=64, h_kv=8, seqlen=2 ** 19),
-               dict(seqlen=257), dict(seqlen=1000), dict(block=64, seqlen=129), dict(seqlen=32768 + 37)):
+               dict(seqlen=257), dict(seqlen=1000), dict(block=64, seqlen=129), dict(seqlen=32768 + 37),
+               dict(granularity="token")):
         p = _p(**kw)
         assert lib.crisp_check_params(ctypes.byref(p)) == 0
         assert lib.crisp_workspace_size(ctypes.byref(p)) > 0
@@ -96,17 +98,17 @@ def test_entry_points_validate_before_launch(lib):
 def test_params_struct_layout_matches_header(lib, tmp_path):
     # 10 int32 + 4 float fields, then the 8-byte seq_lens pointer; the C
     # compiler's view of include/crisp.h must agree with the ctypes mirror
-    assert ctypes.sizeof(B.CrispParams) == 14 * 4 + 8
-    assert B.CrispParams.seq_lens.offset == 56
+    assert ctypes.sizeof(B.CrispParams) == 15 * 4 + 4 + 8        # 4 bytes of padding before the pointer
+    assert B.CrispParams.seq_lens.offset == 64
     src = tmp_path / "layout.c"
     src.write_text(
         '#include <stdio.h>\n#include <stddef.h>\n#include "crisp.h"\n'
         'int main(void) { printf("%zu %zu %zu %zu\\n", sizeof(crisp_params),'
         ' offsetof(crisp_params, seq_lens), offsetof(crisp_params, sm_scale),'
-        ' offsetof(crisp_params, k_min_blocks)); return 0; }\n')
+        ' offsetof(crisp_params, vs_granularity)); return 0; }\n')
     exe = tmp_path / "layout"
     inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
     subprocess.run(["gcc", "-std=c99", "-I", inc, str(src), "-o", str(exe)], check=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
     assert [int(x) for x in out] == [ctypes.sizeof(B.CrispParams), B.CrispParams.seq_lens.offset,
-                                     B.CrispParams.sm_scale.offset, B.CrispParams.k_min_blocks.offset]
+                                     B.CrispParams.sm_scale.offset, B.CrispParams.vs_granularity.offset]

@@ -25,11 +25,13 @@ def _lib():
 
 
 def _check(w, router="cstruct", vs_rule="alpha", alpha=1.0, gamma=0.95, qblocks_fn=None,
-           heads=None, expect_both=False):
+           heads=None, expect_both=False, granularity="tile"):
     q, k, v, meta = make_qkv(w)
-    gpu = PU.run_gpu(w, q, k, v, router=router, vs_rule=vs_rule, alpha=alpha, gamma=gamma)
+    gpu = PU.run_gpu(w, q, k, v, router=router, vs_rule=vs_rule, alpha=alpha, gamma=gamma,
+                     granularity=granularity)
     assert gpu["status"] == 0
-    oprm = PU.oracle_params(w, router=router, vs_rule=vs_rule, alpha=alpha, gamma=gamma)
+    oprm = PU.oracle_params(w, router=router, vs_rule=vs_rule, alpha=alpha, gamma=gamma,
+                            granularity=granularity)
     reps = PU.compare_all(w, q, k, v, gpu, oprm, qblocks_fn=qblocks_fn, heads=heads)
     if expect_both:
         pats = {r["pattern"] for r in reps}
@@ -151,6 +153,35 @@ def test_length_out_of_range_is_reported_and_clamped():
     C.crisp_select(p, qd, kd, pattern, pv, ps, ws)
     assert C.crisp_get_device_status(ws) == -6
     assert C.crisp_get_device_status(ws) == 0
+
+
+# ---- token-granular vertical-slash masks (slash blocks as diagonal bands)
+TOKEN_TINY = Workload("token_tiny", 1, 2, 1, 128, 4096, 128, diffuse_heads=(1,), sink_logit=8.0,
+                      n_vertical=2, recency_peak=9.0, recency_freqs="rope")
+
+
+@pytest.mark.parametrize("alpha", [0.5, 1.0, 2.0])
+def test_token_granularity_tiny(alpha):
+    reps = _check(TOKEN_TINY, alpha=alpha, granularity="token", expect_both=True)
+    assert reps[0]["pattern"] == O.VS
+
+
+@pytest.mark.parametrize("kw", [
+    dict(seqlen=4096 + 77, head_dim=128, h_q=4, h_kv=2),                   # ragged, 77-row last block
+    dict(seqlen=3 * 128 + 1, head_dim=64, h_q=2, h_kv=1),                  # N_b = 4, one-token last block
+    dict(batch=2, seqlen=4096, head_dim=128, h_q=4, h_kv=2, lengths=(3001, 4096)),
+])
+def test_token_granularity_shapes(kw):
+    base = dict(name="token", batch=1, block=128, n_vertical=2, diffuse_frac=0.5, sink_logit=8.0)
+    base.update(kw)
+    _check(Workload(**base), granularity="token")
+
+
+def test_token_granularity_llama_32k():
+    w = WORKLOADS["llama_32k"]
+    reps = _check(w, granularity="token", heads=range(0, 32, 2),
+                  qblocks_fn=lambda b, h: PU.sample_qblocks(w.n_blocks, 3, 5000 + h))
+    assert {r["pattern"] for r in reps} == {O.VS, O.PE}
 
 
 def test_kmin_above_nb():
