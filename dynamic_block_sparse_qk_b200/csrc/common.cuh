@@ -19,7 +19,7 @@ constexpr int kMaxBlocks = 8192;  // N_b limit (selection kernels keep one row i
 // ----------------------------------------------------------------------------
 struct Workspace {
   size_t status;      // int32[64]: [0] status word, [1] first bad index
-  size_t head_cnt;    // uint32[BH][4]: per-head CTA completion counters (proxy, histogram, ties, scores)
+  size_t head_cnt;    // uint32[BH][4]: per-head CTA completion counters (proxy, histogram, ties; one spare)
   size_t stat_m;      // float[BH][Nb][R]   per-row max of a proxy key tile (log2 units)
   size_t stat_lo;     // float[BH][Nb][R]   sum exp2(s-m) over tile columns c <= r
   size_t stat_hi;     // float[BH][Nb][R]   sum exp2(s-m) over tile columns c >  r
@@ -30,6 +30,7 @@ struct Workspace {
   size_t kbar;        // float[B*Hkv][Nb][d] block means of K
   size_t qbar;        // float[BH][Nb][d]    block means of Q (PE heads)
   size_t sel;         // uint8[BH][2][Nb]    selected vertical / slash blocks
+  size_t sel_bits;    // uint32[BH][2][ceil(Nb/32)] the same as bitmasks, plus vertical 0 / slash Nb-1
   size_t abar;        // float[BH][Nb][Nb]   PE estimate divided by N_b
   size_t hist_cnt;    // uint32[BH][4096]    radix-select bucket counts
   size_t hist_sum;    // double[BH][4096]    radix-select bucket sums
@@ -75,7 +76,7 @@ __host__ __device__ inline int proxy_chunk(const crisp_params& p) {
   return int((c + 1) & ~1ll);
 }
 
-enum HeadCounter { kCntProxy = 0, kCntHist = 1, kCntEq = 2, kCntScores = 3 };
+enum HeadCounter { kCntProxy = 0, kCntHist = 1, kCntEq = 2 };   // slot 3 spare
 
 // Tile-list entries in token granularity: key-block id in the low 24 bits,
 // then flags (whole tile; slash blocks N_b-1-delta-1, N_b-1-delta, N_b-delta).
@@ -107,6 +108,7 @@ __host__ __device__ inline Workspace make_workspace(const crisp_params& p) {
   w.kbar = take(BK * nb * d * 4);
   w.qbar = take(BH * nb * d * 4);
   w.sel = take(BH * 2 * nb);
+  w.sel_bits = take(BH * 2 * ((nb + 31) / 32) * 4);
   w.abar = take(BH * nb * nb * 4);
   w.hist_cnt = take(BH * 4096 * 4);
   w.hist_sum = take(BH * 4096 * 8);

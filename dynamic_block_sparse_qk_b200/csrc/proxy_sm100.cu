@@ -57,20 +57,27 @@ struct PxCfg {
   static_assert(2 * (SMEM + 1024) <= 233472, "two CTAs per SM");
 };
 
-// Proxy row max and normaliser of head bh from its nc chunk partials, in
-// chunk order. Out of line so that its addresses are not held in registers
-// through the main loop.
+// Proxy row max and normaliser of head bh from its nc chunk partials: one
+// warp per row, lanes over chunks (fixed order: lane-strided partials, then a
+// butterfly), so the loads of a row are in flight together. Out of line so
+// that its addresses are not held in registers through the main loop.
 __device__ __noinline__ void merge_chunks(const crisp_params& p, void* ws, int bh, int nc, int R) {
   const Workspace W = make_workspace(p);
   const float* cmv = ws_ptr<float>(ws, W.chunk_m) + size_t(bh) * nc * R;
   const float* clv = ws_ptr<float>(ws, W.chunk_l) + size_t(bh) * nc * R;
-  for (int r = threadIdx.x; r < R; r += blockDim.x) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nwarps = blockDim.x >> 5;
+  for (int r = warp; r < R; r += nwarps) {
     float m = -INFINITY;
-    for (int c = 0; c < nc; ++c) m = fmaxf(m, __ldcg(cmv + size_t(c) * R + r));
+    for (int c = lane; c < nc; c += 32) m = fmaxf(m, __ldcg(cmv + size_t(c) * R + r));
+    m = warp_max(m);
     float l = 0.f;
-    for (int c = 0; c < nc; ++c) l += __ldcg(clv + size_t(c) * R + r) * fast_exp2(__ldcg(cmv + size_t(c) * R + r) - m);
-    ws_ptr<float>(ws, W.row_m)[size_t(bh) * R + r] = m;
-    ws_ptr<float>(ws, W.row_l)[size_t(bh) * R + r] = l;
+    for (int c = lane; c < nc; c += 32)
+      l += __ldcg(clv + size_t(c) * R + r) * fast_exp2(__ldcg(cmv + size_t(c) * R + r) - m);
+    l = warp_sum(l);
+    if (lane == 0) {
+      ws_ptr<float>(ws, W.row_m)[size_t(bh) * R + r] = m;
+      ws_ptr<float>(ws, W.row_l)[size_t(bh) * R + r] = l;
+    }
   }
 }
 
@@ -202,26 +209,19 @@ __global__ void __launch_bounds__(kPxThreads, 2)
     float* stat_hi = ws_ptr<float>(ws, W.stat_hi);
     float cm = -INFINITY, cl = 0.f;
 
+    // Columns past this row's causal limit `lim` (only in the last two key
+    // tiles of a sequence) become -inf right after the TMEM load; the max and
+    // sum passes below then need no masking of their own (exp2(-inf) = 0).
+    auto mask_chunk = [&](uint32_t (&a)[32], int ci, int lim) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (ci * 32 + e > lim) a[e] = 0xFF800000u;          // -inf
+    };
     // exp2(s * sl2 - mx) summed over one 32-column chunk into lo (columns <= pr)
     // and hi (columns > pr); `ci` is the chunk index inside its key tile.
-    // `lim` is the last key column this row may see in the tile (causal
-    // limit); only the last two tiles of a sequence (`masked`) have one below
-    // the tile width, and there every column is tested on its own.
-    auto chunk_sums = [&](const uint32_t (&a)[32], int ci, bool masked, int lim, float mx, uint64_t& lo2,
-                          uint64_t& hi2) {
+    auto chunk_sums = [&](const uint32_t (&a)[32], int ci, float mx, uint64_t& lo2, uint64_t& hi2) {
       const uint64_t nm2 = pack_f32x2(-mx, -mx);
-      if (masked) {
-        float lo = 0.f, hi = 0.f;
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = ci * 32 + e;
-          const float ex = c <= lim ? fast_exp2(fmaf(__uint_as_float(a[e]), sl2, -mx)) : 0.f;
-          if (c <= pr) lo += ex;
-          else hi += ex;
-        }
-        lo2 = add_f32x2(lo2, pack_f32x2(lo, 0.f));
-        hi2 = add_f32x2(hi2, pack_f32x2(hi, 0.f));
-      } else if (ci != mixc) {
+      if (ci != mixc) {
         uint64_t acc2[2] = {pack_f32x2(0.f, 0.f), pack_f32x2(0.f, 0.f)};
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
@@ -245,19 +245,13 @@ __global__ void __launch_bounds__(kPxThreads, 2)
         hi2 = add_f32x2(hi2, pack_f32x2(hi, 0.f));
       }
     };
-    // max over one chunk (raw scores), visible columns only
-    auto chunk_max = [&](const uint32_t (&a)[32], int ci, bool masked, int lim, float mx) -> float {
-      if (!masked) {
-        float m2[2] = {mx, -INFINITY};
+    // max over one chunk (raw scores)
+    auto chunk_max = [&](const uint32_t (&a)[32], float mx) -> float {
+      float m2[2] = {mx, -INFINITY};
 #pragma unroll
-        for (int e = 0; e < 32; e += 2)
-          m2[(e >> 1) & 1] = max3f(m2[(e >> 1) & 1], __uint_as_float(a[e]), __uint_as_float(a[e + 1]));
-        return fmaxf(m2[0], m2[1]);
-      }
-#pragma unroll
-      for (int e = 0; e < 32; ++e)
-        if (ci * 32 + e <= lim) mx = fmaxf(mx, __uint_as_float(a[e]));
-      return mx;
+      for (int e = 0; e < 32; e += 2)
+        m2[(e >> 1) & 1] = max3f(m2[(e >> 1) & 1], __uint_as_float(a[e]), __uint_as_float(a[e + 1]));
+      return fmaxf(m2[0], m2[1]);
     };
     // A row with no visible key in the tile (possible in a partial last block)
     // stores max -inf and zero sums and leaves the running (max, sum) alone.
@@ -300,14 +294,17 @@ __global__ void __launch_bounds__(kPxThreads, 2)
           }
           const int kb = kbs + ks;
           if (kb < kb1) {
-            const bool masked = kb >= nbv - 2;
-            const int lim = t_row - kb * R;
-            float mx = chunk_max(a0, 0, masked, lim, -INFINITY);
-            mx = chunk_max(a1, 1, masked, lim, mx) * sl2;
+            if (kb >= nbv - 2) {                         // causal limit inside the tile
+              const int lim = t_row - kb * R;
+              mask_chunk(a0, 0, lim);
+              mask_chunk(a1, 1, lim);
+            }
+            float mx = chunk_max(a0, -INFINITY);
+            mx = chunk_max(a1, mx) * sl2;
             uint64_t lo2 = pack_f32x2(0.f, 0.f), hi2 = pack_f32x2(0.f, 0.f);
             if (mx != -INFINITY) {
-              chunk_sums(a0, 0, masked, lim, mx, lo2, hi2);
-              chunk_sums(a1, 1, masked, lim, mx, lo2, hi2);
+              chunk_sums(a0, 0, mx, lo2, hi2);
+              chunk_sums(a1, 1, mx, lo2, hi2);
             }
             finish_tile(kb, mx, lo2, hi2);
           }
@@ -315,24 +312,32 @@ __global__ void __launch_bounds__(kPxThreads, 2)
       } else {
         // one 128-key tile: a max pass and a sum pass over two pairs of chunks
         const int kb = kbs;
-        const bool masked = kb >= nbv - 2;
+        const bool masked = kb >= nbv - 2;               // causal limit inside the tile
         const int lim = t_row - kb * R;
         tmem_ld32(tS, a0);
         tmem_ld32(tS + 32, a1);
         tmem_wait_ld();
-        float mx = chunk_max(a0, 0, masked, lim, -INFINITY);
-        mx = chunk_max(a1, 1, masked, lim, mx);
+        if (masked) {
+          mask_chunk(a0, 0, lim);
+          mask_chunk(a1, 1, lim);
+        }
+        float mx = chunk_max(a0, -INFINITY);
+        mx = chunk_max(a1, mx);
         uint32_t a2[32], a3[32];
         tmem_ld32(tS + 64, a2);
         tmem_ld32(tS + 96, a3);
         tmem_wait_ld();
-        mx = chunk_max(a2, 2, masked, lim, mx);
-        mx = chunk_max(a3, 3, masked, lim, mx) * sl2;
+        if (masked) {
+          mask_chunk(a2, 2, lim);
+          mask_chunk(a3, 3, lim);
+        }
+        mx = chunk_max(a2, mx);
+        mx = chunk_max(a3, mx) * sl2;
         uint64_t lo2 = pack_f32x2(0.f, 0.f), hi2 = pack_f32x2(0.f, 0.f);
         const bool any = mx != -INFINITY;
         if (any) {
-          chunk_sums(a2, 2, masked, lim, mx, lo2, hi2);
-          chunk_sums(a3, 3, masked, lim, mx, lo2, hi2);
+          chunk_sums(a2, 2, mx, lo2, hi2);
+          chunk_sums(a3, 3, mx, lo2, hi2);
         }
         tmem_ld32(tS, a0);
         tmem_ld32(tS + 32, a1);
@@ -340,9 +345,13 @@ __global__ void __launch_bounds__(kPxThreads, 2)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::B_SFREE + grp));
+        if (masked) {
+          mask_chunk(a0, 0, lim);
+          mask_chunk(a1, 1, lim);
+        }
         if (any) {
-          chunk_sums(a0, 0, masked, lim, mx, lo2, hi2);
-          chunk_sums(a1, 1, masked, lim, mx, lo2, hi2);
+          chunk_sums(a0, 0, mx, lo2, hi2);
+          chunk_sums(a1, 1, mx, lo2, hi2);
         }
         finish_tile(kb, mx, lo2, hi2);
       }

@@ -18,117 +18,124 @@ namespace crisp {
 
 // p_v[kb] = (1/R) sum_r w(r,kb) (lo+hi);  p_s[kb] = (1/R) sum_r [w(r,kb) lo(kb) + w(r,kb-1) hi(kb-1)]
 // with w(r,kb) = exp2(m(r,kb) - m_r) / l_r. One warp per key block. With the
-// C_struct router the last CTA of a head also routes it (Eq. 2:
-// C_struct = p_v[0] + p_v[N_b-1], VS iff >= tau_proxy).
+// C_struct router the first warp of the first CTA of a head also routes it
+// (Eq. 2: C_struct = p_v[0] + p_v[N_b-1], VS iff >= tau_proxy), recomputing
+// p_v[N_b-1] with the same arithmetic as the warp that stores it.
 __global__ void proxy_scores_kernel(crisp_params p, void* ws, float* __restrict__ p_v,
                                     float* __restrict__ p_s, int32_t* __restrict__ pattern,
                                     float* __restrict__ score) {
-  __shared__ int last;
   const Workspace W = make_workspace(p);
   const int R = p.block, nb = n_blocks(p);
   const int bh = blockIdx.y;
   const int nbv = (seq_len(p, bh / p.h_q) + R - 1) / R;   // this sequence's blocks
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kb = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (kb >= nbv && kb < nb && lane == 0) {          // past the end of a shorter sequence
-    p_v[size_t(bh) * nb + kb] = 0.f;
-    p_s[size_t(bh) * nb + kb] = 0.f;
-  }
-  if (kb < nbv) {
-    const float* sm = ws_ptr<float>(ws, W.stat_m) + size_t(bh) * nb * R;
-    const float* slo = ws_ptr<float>(ws, W.stat_lo) + size_t(bh) * nb * R;
-    const float* shi = ws_ptr<float>(ws, W.stat_hi) + size_t(bh) * nb * R;
-    const float* rm = ws_ptr<float>(ws, W.row_m) + size_t(bh) * R;
-    const float* rl = ws_ptr<float>(ws, W.row_l) + size_t(bh) * R;
-    float sv = 0.f, ss = 0.f;
+  const float* sm = ws_ptr<float>(ws, W.stat_m) + size_t(bh) * nb * R;
+  const float* slo = ws_ptr<float>(ws, W.stat_lo) + size_t(bh) * nb * R;
+  const float* shi = ws_ptr<float>(ws, W.stat_hi) + size_t(bh) * nb * R;
+  const float* rm = ws_ptr<float>(ws, W.row_m) + size_t(bh) * R;
+  const float* rl = ws_ptr<float>(ws, W.row_l) + size_t(bh) * R;
+  auto block_scores = [&](int j, float& sv, float& ss) {
+    sv = 0.f;
+    ss = 0.f;
     for (int r = lane; r < R; r += 32) {
       const float il = 1.f / rl[r];
-      const size_t o = size_t(kb) * R + r;
+      const size_t o = size_t(j) * R + r;
       const float w = fast_exp2(sm[o] - rm[r]) * il;
       sv += w * (slo[o] + shi[o]);
       ss += w * slo[o];
-      if (kb > 0) {
+      if (j > 0) {
         const size_t o1 = o - R;
         ss += fast_exp2(sm[o1] - rm[r]) * il * shi[o1];
       }
     }
-    sv = warp_sum(sv);
-    ss = warp_sum(ss);
+    sv = warp_sum(sv) / float(R);
+    ss = warp_sum(ss) / float(R);
+  };
+  float sv = 0.f, ss = 0.f;
+  if (kb < nbv) {
+    block_scores(kb, sv, ss);
     if (lane == 0) {
-      p_v[size_t(bh) * nb + kb] = sv / float(R);
-      p_s[size_t(bh) * nb + kb] = ss / float(R);
+      p_v[size_t(bh) * nb + kb] = sv;
+      p_s[size_t(bh) * nb + kb] = ss;
+    }
+  } else if (kb < nb && lane == 0) {                 // past the end of a shorter sequence
+    p_v[size_t(bh) * nb + kb] = 0.f;
+    p_s[size_t(bh) * nb + kb] = 0.f;
+  }
+  if (p.router != CRISP_ROUTER_JSD && kb == 0) {     // routed by route_kernel after K pooling otherwise
+    float sv_last, ss_last;
+    block_scores(nbv - 1, sv_last, ss_last);
+    if (lane == 0) {
+      const float c = sv + sv_last;
+      score[bh] = c;
+      pattern[bh] = (c >= p.tau_proxy) ? CRISP_PATTERN_VS : CRISP_PATTERN_PE;
     }
   }
-  if (p.router == CRISP_ROUTER_JSD) return;     // routed by route_kernel after K pooling
-  __threadfence();
-  __syncthreads();
-  uint32_t* cnt = ws_ptr<uint32_t>(ws, W.head_cnt) + size_t(bh) * 4 + kCntScores;
-  if (threadIdx.x == 0) last = atomicAdd(cnt, 1u) == gridDim.x - 1;
-  __syncthreads();
-  if (!last || threadIdx.x != 0) return;
-  __threadfence();
-  const float c = __ldcg(p_v + size_t(bh) * nb) + __ldcg(p_v + size_t(bh) * nb + nbv - 1);
-  score[bh] = c;
-  pattern[bh] = (c >= p.tau_proxy) ? CRISP_PATTERN_VS : CRISP_PATTERN_PE;
-  *cnt = 0u;
 }
 
 // ---------------------------------------------------------------------------
-// Block-mean pooling (Algorithm 4 line 3; Algorithm 5 line 3): one CTA per
-// (head, block); 16-byte loads, rows split across thread groups, smem reduce.
-// One launch covers K and Q: rows y < nk of the grid are K heads (skipped
-// unless a query head of the group is PE, or pattern == NULL), the rest Q
-// heads (only PE heads).
+// Block-mean pooling (Algorithm 4 line 3; Algorithm 5 line 3): a block of
+// one head per CTA step (16-byte loads, rows split across thread groups,
+// smem reduce), grid-stride over blocks. One launch covers K and Q: heads
+// y < nk are K heads (skipped unless a query head of the group is PE, or
+// pattern == NULL), the next nq are Q heads (only PE heads).
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restrict__ k,
                                                    const __nv_bfloat16* __restrict__ q,
-                                                   crisp_params p, const int32_t* pattern, int nk,
+                                                   crisp_params p, const int32_t* pattern, int nk, int nq,
                                                    float* __restrict__ kbar, float* __restrict__ qbar) {
   constexpr int CPR = D / 8;
   constexpr int RPP = 256 / CPR;   // rows per pass
   __shared__ float part[RPP][D];
   const int R = p.block, nb = n_blocks(p);
-  const int kb = blockIdx.x;
-  const bool is_k = int(blockIdx.y) < nk;
-  const int hh = is_k ? int(blockIdx.y) : int(blockIdx.y) - nk;
-  const int len = seq_len(p, hh / (is_k ? p.h_kv : p.h_q));
-  const int rows = min(R, len - kb * R);            // a partial last block averages what it holds
-  if (rows <= 0) return;
-  const __nv_bfloat16* x = is_k ? k : q;
-  float* out = is_k ? kbar : qbar;
-  if (pattern) {
-    if (!is_k) {
-      if (pattern[hh] != CRISP_PATTERN_PE) return;
-    } else {
-      const int g = p.h_q / p.h_kv;
-      const int b = hh / p.h_kv, hk = hh % p.h_kv;
-      bool any = false;
-      for (int i = 0; i < g; ++i) any |= pattern[b * p.h_q + hk * g + i] == CRISP_PATTERN_PE;
-      if (!any) return;
-    }
-  }
   const int tid = threadIdx.x, c = tid % CPR, rg = tid / CPR;
-  const __nv_bfloat16* src = x + (size_t(hh) * p.seqlen + size_t(kb) * R) * D;
-  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  for (int row = rg; row < rows; row += RPP) {
-    const uint4 u = *reinterpret_cast<const uint4*>(src + size_t(row) * D + c * 8);
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __bfloat1622float2(h2[i]);
-      acc[2 * i] += f.x;
-      acc[2 * i + 1] += f.y;
+  // Grid-stride over (head, block): a head nobody needs is skipped once per
+  // CTA instead of launching a CTA per block of it.
+  for (int hy = 0; hy < nk + nq; ++hy) {
+    const bool is_k = hy < nk;
+    const int hh = is_k ? hy : hy - nk;
+    if (pattern) {
+      bool any = false;
+      if (!is_k) {
+        any = pattern[hh] == CRISP_PATTERN_PE;
+      } else {
+        const int g = p.h_q / p.h_kv;
+        const int b = hh / p.h_kv, hk = hh % p.h_kv;
+        for (int i = 0; i < g; ++i) any |= pattern[b * p.h_q + hk * g + i] == CRISP_PATTERN_PE;
+      }
+      if (!any) continue;
     }
-  }
+    const int len = seq_len(p, hh / (is_k ? p.h_kv : p.h_q));
+    const int nbv = (len + R - 1) / R;
+    const __nv_bfloat16* x = is_k ? k : q;
+    float* out = is_k ? kbar : qbar;
+    for (int kb = blockIdx.x; kb < nbv; kb += gridDim.x) {
+      const int rows = min(R, len - kb * R);         // a partial last block averages what it holds
+      const __nv_bfloat16* src = x + (size_t(hh) * p.seqlen + size_t(kb) * R) * D;
+      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int row = rg; row < rows; row += RPP) {
+        const uint4 u = *reinterpret_cast<const uint4*>(src + size_t(row) * D + c * 8);
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) part[rg][c * 8 + i] = acc[i];
-  __syncthreads();
-  for (int dd = tid; dd < D; dd += 256) {
-    float s = 0.f;
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = __bfloat1622float2(h2[i]);
+          acc[2 * i] += f.x;
+          acc[2 * i + 1] += f.y;
+        }
+      }
 #pragma unroll
-    for (int i = 0; i < RPP; ++i) s += part[i][dd];
-    out[(size_t(hh) * nb + kb) * D + dd] = s / float(rows);
+      for (int i = 0; i < 8; ++i) part[rg][c * 8 + i] = acc[i];
+      __syncthreads();
+      for (int dd = tid; dd < D; dd += 256) {
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < RPP; ++i) s += part[i][dd];
+        out[(size_t(hh) * nb + kb) * D + dd] = s / float(rows);
+      }
+      __syncthreads();
+    }
   }
 }
 
@@ -217,13 +224,13 @@ cudaError_t launch_pool(const crisp_params& p, const void* k, const void* q, int
                         const int32_t* pattern, float* kbar, float* qbar, cudaStream_t st) {
   if (nk + nq == 0) return cudaSuccess;
   const int nb = n_blocks(p);
-  dim3 grid(nb, nk + nq);
+  const unsigned grid = unsigned(min(nb, 4 * 148));
   const auto* kk = static_cast<const __nv_bfloat16*>(k);
   const auto* qq = static_cast<const __nv_bfloat16*>(q);
   if (p.head_dim == 64)
-    pool_kernel<64><<<grid, 256, 0, st>>>(kk, qq, p, pattern, nk, kbar, qbar);
+    pool_kernel<64><<<grid, 256, 0, st>>>(kk, qq, p, pattern, nk, nq, kbar, qbar);
   else
-    pool_kernel<128><<<grid, 256, 0, st>>>(kk, qq, p, pattern, nk, kbar, qbar);
+    pool_kernel<128><<<grid, 256, 0, st>>>(kk, qq, p, pattern, nk, nq, kbar, qbar);
   return cudaGetLastError();
 }
 
@@ -233,7 +240,7 @@ cudaError_t run_route(const crisp_params& p, const void* q, const void* k, void*
   const int nb = n_blocks(p);
   const int BH = p.batch * p.h_q;
   // proxy statistics (+ row merge in the last CTA of each head), block
-  // scores (+ C_struct route in the last CTA of each head)
+  // scores (+ C_struct route by the warp that computes p_v[0])
   cudaError_t e = run_proxy_stats(p, q, k, ws, st);
   if (e != cudaSuccess) return e;
   proxy_scores_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, ws, p_v, p_s, pattern, score);

@@ -53,6 +53,19 @@ __global__ void __launch_bounds__(1024) vs_select_kernel(crisp_params p, const i
   for (int j = tid; j < nb; j += 1024) pv[j] = src[j];
   if (tid == 0) { cnt_s = 0; kcut_s = nb; }
   __syncthreads();
+  // The selection as bitmasks (one bit per block, the always-kept vertical
+  // block 0 / slash block N_b-1 included) for the tile builder.
+  auto write_bits = [&]() {
+    __syncthreads();                                     // this CTA's sel[] stores are visible
+    const int nw = (nbs + 31) / 32, lane = tid & 31;
+    uint32_t* bits = ws_ptr<uint32_t>(ws, W.sel_bits) + (size_t(bh) * 2 + dir) * nw;
+    const int always = dir == 0 ? 0 : nb - 1;
+    for (int w = tid >> 5; w < nw; w += 32) {
+      const int j = w * 32 + lane;
+      const unsigned m = __ballot_sync(0xffffffffu, j < nb && (j == always || sel[j] != 0));
+      if (lane == 0) bits[w] = m;
+    }
+  };
   auto rank_of = [&](int j) {
     const float x = pv[j];
     int rk = 0;
@@ -97,9 +110,10 @@ __global__ void __launch_bounds__(1024) vs_select_kernel(crisp_params p, const i
     k = min(max(cnt, p.k_min_blocks), nb);
     if (k == cnt) {
       for (int j = tid; j < nb; j += 1024) sel[j] = pv[j] > thr;
-      return;
+    } else {
+      for (int j = tid; j < nb; j += 1024) sel[j] = rank_of(j) < k;
     }
-    for (int j = tid; j < nb; j += 1024) sel[j] = rank_of(j) < k;
+    write_bits();
     return;
   }
   // GAMMA (Algorithm 6).
@@ -127,11 +141,13 @@ __global__ void __launch_bounds__(1024) vs_select_kernel(crisp_params p, const i
   __syncthreads();
   k = min(max(kcut_s, p.k_min_blocks), nb);
   for (int j = tid; j < nb; j += 1024) sel[j] = rank_of(j) < k;
+  write_bits();
 }
 
 // ---------------------------------------------------------------------------
 // PE estimate (Algorithm 4 line 4): logits of Q_bar K_bar^T for kb <= qb,
-// 64x64 tiles per CTA, fp32 FMA; written in log2 units into abar together
+// 64x64 tiles (grid-stride over PE heads and tiles), fp32 FMA; written in
+// log2 units into abar together
 // with per-(row, tile) max / sum partials. Then a row pass normalises and
 // divides by N_b (Algorithm 4 line 6: the total of N_b causal rows is N_b).
 // ---------------------------------------------------------------------------
@@ -144,70 +160,80 @@ __global__ void __launch_bounds__(256) pe_logits_kernel(crisp_params p, const in
   __shared__ float rmax[T][17], rsum[T][17];
   const Workspace W = make_workspace(p);
   const int nb = n_blocks(p);                               // stride
-  const int bh = blockIdx.z;
-  if (pattern[bh] != CRISP_PATTERN_PE) return;
-  const int nbv = (seq_len(p, bh / p.h_q) + p.block - 1) / p.block;   // this sequence's blocks
-  const int tq = blockIdx.y, tk = blockIdx.x;
-  if (tk > tq || tq * 64 >= nbv) return;
-  const int b = bh / p.h_q, h = bh % p.h_q, hk = h / (p.h_q / p.h_kv);
-  const float* qbar = ws_ptr<float>(ws, W.qbar) + size_t(bh) * nb * D;
-  const float* kbar = ws_ptr<float>(ws, W.kbar) + (size_t(b) * p.h_kv + hk) * nb * D;
-  float* abar = ws_ptr<float>(ws, W.abar) + size_t(bh) * nb * nb;
-  const float sl2 = (p.sm_scale > 0.f ? p.sm_scale : rsqrtf(float(D))) * kLog2e;
-  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;   // 4x4 micro-tile per thread
-  float acc[4][4] = {};
-  for (int k0 = 0; k0 < D; k0 += KC) {
-    for (int i = tid; i < T * KC; i += 256) {
-      const int r = i / KC, c = i % KC;
-      const int qr = tq * T + r, kr = tk * T + r;
-      qs[c][r] = qr < nbv ? qbar[size_t(qr) * D + k0 + c] : 0.f;
-      kst[c][r] = kr < nbv ? kbar[size_t(kr) * D + k0 + c] : 0.f;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int c = 0; c < KC; ++c) {
-      float a[4], bb[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) { a[i] = qs[c][ty * 4 + i]; bb[i] = kst[c][tx * 4 + i]; }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-  // write logits (log2 units) and per-row partial max / sum over this tile
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int qb = tq * T + ty * 4 + i;
-    float mx = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int kb = tk * T + tx * 4 + j;
-      const bool ok = qb < nbv && kb <= qb;
-      acc[i][j] = ok ? acc[i][j] * sl2 : -INFINITY;
-      if (ok) abar[size_t(qb) * nb + kb] = acc[i][j];
-      mx = fmaxf(mx, acc[i][j]);
-    }
-    float s = 0.f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) s += (acc[i][j] == -INFINITY) ? 0.f : exp2f(acc[i][j] - mx);
-    rmax[ty * 4 + i][tx] = mx;
-    rsum[ty * 4 + i][tx] = s;
-  }
-  __syncthreads();
-  if (tid < T) {
-    const int qb = tq * T + tid;
-    if (qb < nbv) {
-      float mx = -INFINITY;
-      for (int j = 0; j < 16; ++j) mx = fmaxf(mx, rmax[tid][j]);
-      float s = 0.f;
-      for (int j = 0; j < 16; ++j)
-        if (rmax[tid][j] != -INFINITY) s += rsum[tid][j] * exp2f(rmax[tid][j] - mx);
-      const int ntile = (nb + T - 1) / T;
-      // partials reuse the proxy statistic regions (free once routing is done)
-      ws_ptr<float>(ws, W.stat_m)[(size_t(bh) * nb + qb) * ntile + tk] = mx;
-      ws_ptr<float>(ws, W.stat_lo)[(size_t(bh) * nb + qb) * ntile + tk] = s;
+  const int BH = p.batch * p.h_q;
+  // Grid-stride over (PE head, lower-triangle 64x64 tile): heads that are
+  // not PE cost one check per CTA.
+  for (int bh = 0; bh < BH; ++bh) {
+    if (pattern[bh] != CRISP_PATTERN_PE) continue;
+    const int nbv = (seq_len(p, bh / p.h_q) + p.block - 1) / p.block;   // this sequence's blocks
+    const int ntq = (nbv + T - 1) / T;
+    for (int tt = blockIdx.x; tt < ntq * (ntq + 1) / 2; tt += gridDim.x) {
+      int tq = int((sqrtf(8.f * float(tt) + 1.f) - 1.f) * 0.5f);
+      while ((tq + 1) * (tq + 2) / 2 <= tt) ++tq;
+      while (tq * (tq + 1) / 2 > tt) --tq;
+      const int tk = tt - tq * (tq + 1) / 2;
+      const int b = bh / p.h_q, h = bh % p.h_q, hk = h / (p.h_q / p.h_kv);
+      const float* qbar = ws_ptr<float>(ws, W.qbar) + size_t(bh) * nb * D;
+      const float* kbar = ws_ptr<float>(ws, W.kbar) + (size_t(b) * p.h_kv + hk) * nb * D;
+      float* abar = ws_ptr<float>(ws, W.abar) + size_t(bh) * nb * nb;
+      const float sl2 = (p.sm_scale > 0.f ? p.sm_scale : rsqrtf(float(D))) * kLog2e;
+      const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;   // 4x4 micro-tile per thread
+      float acc[4][4] = {};
+      for (int k0 = 0; k0 < D; k0 += KC) {
+        for (int i = tid; i < T * KC; i += 256) {
+          const int r = i / KC, c = i % KC;
+          const int qr = tq * T + r, kr = tk * T + r;
+          qs[c][r] = qr < nbv ? qbar[size_t(qr) * D + k0 + c] : 0.f;
+          kst[c][r] = kr < nbv ? kbar[size_t(kr) * D + k0 + c] : 0.f;
+        }
+        __syncthreads();
+    #pragma unroll 8
+        for (int c = 0; c < KC; ++c) {
+          float a[4], bb[4];
+    #pragma unroll
+          for (int i = 0; i < 4; ++i) { a[i] = qs[c][ty * 4 + i]; bb[i] = kst[c][tx * 4 + i]; }
+    #pragma unroll
+          for (int i = 0; i < 4; ++i)
+    #pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], bb[j], acc[i][j]);
+        }
+        __syncthreads();
+      }
+      // write logits (log2 units) and per-row partial max / sum over this tile
+    #pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int qb = tq * T + ty * 4 + i;
+        float mx = -INFINITY;
+    #pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int kb = tk * T + tx * 4 + j;
+          const bool ok = qb < nbv && kb <= qb;
+          acc[i][j] = ok ? acc[i][j] * sl2 : -INFINITY;
+          if (ok) abar[size_t(qb) * nb + kb] = acc[i][j];
+          mx = fmaxf(mx, acc[i][j]);
+        }
+        float s = 0.f;
+    #pragma unroll
+        for (int j = 0; j < 4; ++j) s += (acc[i][j] == -INFINITY) ? 0.f : exp2f(acc[i][j] - mx);
+        rmax[ty * 4 + i][tx] = mx;
+        rsum[ty * 4 + i][tx] = s;
+      }
+      __syncthreads();
+      if (tid < T) {
+        const int qb = tq * T + tid;
+        if (qb < nbv) {
+          float mx = -INFINITY;
+          for (int j = 0; j < 16; ++j) mx = fmaxf(mx, rmax[tid][j]);
+          float s = 0.f;
+          for (int j = 0; j < 16; ++j)
+            if (rmax[tid][j] != -INFINITY) s += rsum[tid][j] * exp2f(rmax[tid][j] - mx);
+          const int ntile = (nb + T - 1) / T;
+          // partials reuse the proxy statistic regions (free once routing is done)
+          ws_ptr<float>(ws, W.stat_m)[(size_t(bh) * nb + qb) * ntile + tk] = mx;
+          ws_ptr<float>(ws, W.stat_lo)[(size_t(bh) * nb + qb) * ntile + tk] = s;
+        }
+      }
+      __syncthreads();                                      // rmax / rsum are reused
     }
   }
 }
@@ -485,8 +511,9 @@ __global__ void __launch_bounds__(256) build_tiles_kernel(crisp_params p, const 
   // j + len-1-t = (nb-1-delta) B + s + (c - r) with s = (len-1) mod B and
   // c - r over [-(rows(qb)-1), cols(kb)-1] (off the diagonal) or
   // [-(rows(qb)-1), 0] (on it); so the blocks nb-1-delta + {-1, 0, +1}
-  // with the two ends decided by the signs below. For len a multiple of B
-  // this is {nb-1-delta, nb-delta}: offsets delta and delta-1.
+  // with the two ends decided by the signs below: -1 when some row of qb
+  // lies past s (lo_ext), +1 off the diagonal when s >= 1. For len a
+  // multiple of B this is {nb-1-delta, nb-delta}: offsets delta and delta-1.
   const int s_res = (len - 1) % B;
   const int rows_q = min(B, len - qb * B);
   const bool lo_ext = s_res - (rows_q - 1) < 0;
@@ -503,15 +530,53 @@ __global__ void __launch_bounds__(256) build_tiles_kernel(crisp_params p, const 
       if (slash_on(nb - 1 - (qb - kb) + e)) v |= 1 << (kTileSlashShift + e + 1);
     return v;
   };
-  auto slash_hit = [&](int kb) -> bool {
-    const int dlt = qb - kb;
-    const int vmax = dlt >= 1 ? B - 1 : 0;                  // key blocks before qb are full
-    const int lo = nb - 1 - dlt - (lo_ext ? 1 : 0);
-    const int hi = nb - 1 - dlt + (s_res + vmax >= B ? 1 : 0);
-    for (int jb = lo; jb <= hi; ++jb)
-      if (slash_on(jb)) return true;
-    return false;
-  };
+
+  if (vs) {
+    // Vertical-slash row from the selection bitmasks, 32 key blocks per lane
+    // word: kb is active iff it is a selected vertical block, or a selected
+    // slash block jb = kb + c0 + t meets the tile, c0 = nb-1-qb and
+    // t in [-1 if lo_ext, +1 if the bands reach the next block] (the slash
+    // rule above, inverted).
+    const int nw = (nbs + 31) / 32;
+    const uint32_t* vwd = ws_ptr<uint32_t>(ws, W.sel_bits) + size_t(bh) * 2 * nw;
+    const uint32_t* swd = vwd + nw;
+    const int c0 = nb - 1 - qb;
+    const bool up = s_res >= 1;                              // bands of full blocks reach jb + 1
+    auto sword = [&](int wd, int sh) -> uint32_t {           // word wd of (S >> sh)
+      const int base = wd * 32 + sh;
+      const int q = base >> 5, rr = base & 31;
+      const uint32_t lo = (q >= 0 && q < nw) ? swd[q] : 0u;
+      const uint32_t hi = (q + 1 >= 0 && q + 1 < nw) ? swd[q + 1] : 0u;
+      return rr ? (lo >> rr) | (hi << (32 - rr)) : lo;
+    };
+    const int nwq = (qb >> 5) + 1;                           // words holding kb <= qb
+    int count = 0;
+    for (int w0 = 0; w0 < nwq; w0 += 32) {
+      const int wd = w0 + lane;
+      uint32_t m = 0;
+      if (wd < nwq) {
+        m = vwd[wd] | sword(wd, c0);
+        if (lo_ext) m |= sword(wd, c0 - 1);
+        if (up) m |= sword(wd, c0 + 1);
+        if (wd == nwq - 1 && (qb & 31) != 31) m &= (2u << (qb & 31)) - 1u;   // kb <= qb
+      }
+      const int c = __popc(m);
+      int pre = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, pre, o);
+        if (lane >= o) pre += v;
+      }
+      int pos = count + pre - c;
+      for (uint32_t mm = m; mm; mm &= mm - 1) idx[pos++] = tile_entry(wd * 32 + __ffs(mm) - 1);
+      if (mrow && wd < nwq)
+        for (int i = 0; i < 32 && wd * 32 + i < nbs; ++i) mrow[wd * 32 + i] = (m >> i) & 1u;
+      count += __shfl_sync(0xffffffffu, pre, 31);
+    }
+    for (int j = nwq * 32 + lane; mrow && j < nbs; j += 32) mrow[j] = 0;
+    if (lane == 0) tile_cnt[size_t(bh) * nbs + qb] = count;
+    return;
+  }
   int count = 0;
   uint32_t eq_seen = eq_before;
   for (int base = 0; base <= qb; base += 128) {
@@ -523,21 +588,17 @@ __global__ void __launch_bounds__(256) build_tiles_kernel(crisp_params p, const 
       const int kb = base + lane * 4 + i;
       bool on = false;
       isq[i] = false;
-      if (kb <= qb) {
-        if (vs) {
-          on = kb == 0 || sv[kb] || slash_hit(kb);
-        } else {
-          on = kb == 0 || kb == qb || st.all;
-          if (!st.all) {
-            const float v = arow[kb];
-            if (v > tv) on = true;
-            else if (v == tv) { isq[i] = true; ++neq; }
-          }
+      if (kb <= qb) {                                      // PE row (VS rows returned above)
+        on = kb == 0 || kb == qb || st.all;
+        if (!st.all) {
+          const float v = arow[kb];
+          if (v > tv) on = true;
+          else if (v == tv) { isq[i] = true; ++neq; }
         }
       }
       f[i] = on;
     }
-    if (!vs && !st.all) {
+    if (!st.all) {
       // rank of this lane's equal entries among all equal entries in flat order
       uint32_t pre = neq;
 #pragma unroll
@@ -602,7 +663,7 @@ cudaError_t run_select(const crisp_params& p, const void* q, const void* k, cons
   if (e != cudaSuccess) return e;
   {
     const int nt = (nb + 63) / 64;
-    dim3 grid(nt, nt, BH);
+    const unsigned grid = unsigned(min(nt * (nt + 1) / 2 * BH, 4 * 148));
     if (p.head_dim == 64) pe_logits_kernel<64><<<grid, 256, 0, st>>>(p, pattern, ws);
     else pe_logits_kernel<128><<<grid, 256, 0, st>>>(p, pattern, ws);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
