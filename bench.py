@@ -358,9 +358,10 @@ def run_sweep(args, out_path):
                     s = out["s"]
                     out["a"] = C.crisp_sparse_prefill(p, q, k, v, s[1], s[2], ws, want_lse=False)
 
-                t_route = timed(route)
-                t_select = timed(select)
-                t_attend = timed(attend)
+                with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+                    t_route = timed(route)
+                    t_select = timed(select)
+                    t_attend = timed(attend)
                 pattern, tcnt = out["r"][0], out["s"][2]
                 nb = w.n_blocks
                 causal = p.batch * p.h_q * nb * (nb + 1) // 2
@@ -373,7 +374,8 @@ def run_sweep(args, out_path):
                        "vs_heads": int((pattern == 0).sum()), "heads": p.batch * p.h_q,
                        "cstruct_jsd_agreement": round(float((pattern == pat_j).float().mean()), 4),
                        "attend_tflops": round(int(tcnt.sum()) * 4 * w.block ** 2 * w.head_dim
-                                              / (t_attend * 1e-3) / 1e12, 1)}
+                                              / (t_attend * 1e-3) / 1e12, 1),
+                       "clocks": clk.summary()}
                 with open(out_path, "a") as fo:
                     fo.write(json.dumps(rec) + "\n")
                 print(json.dumps(rec), flush=True)
