@@ -275,7 +275,7 @@ __device__ inline void level_geom(int level, int& shift, int& nbk) {
 
 // The highest bucket whose descending cumulative sum (above_sum + buckets
 // above + itself) reaches gamma; run by the 256 threads of the last histogram
-// CTA of a head. suf: 256 doubles of shared scratch, ctl: 2 ints.
+// CTA of a head. suf: 257 doubles of shared scratch, ctl: 2 ints.
 __device__ void pe_find(const crisp_params& p, PeState* stp, uint32_t* gc, double* gs, int level,
                         double* suf, int* ctl) {
   int shift, nbk;
@@ -301,14 +301,20 @@ __device__ void pe_find(const crisp_params& p, PeState* stp, uint32_t* gc, doubl
   const double g = double(p.gamma);
   const double above0 = stp->above_sum;
   double run = above0 + (tid > 0 ? suf[tid - 1] : 0.0);
+  int cand = -1;
+  double cand_above = 0.0;                 // sum strictly above this thread's candidate bucket
   for (int i = 0; i < per; ++i) {
     const int bk = nbk - 1 - (tid * per + i);
     const double v = __ldcg(gs + bk);
-    if (run + v >= g) { atomicMax(&best, bk); break; }
+    if (run + v >= g) { cand = bk; cand_above = run; atomicMax(&best, bk); break; }
     run += v;
   }
   __syncthreads();
-  // Recompute the sum strictly above the chosen bucket (single thread, exact order).
+  // the owner of the chosen bucket (ranges are disjoint: exactly one thread)
+  // hands over the sum strictly above it
+  double* above_s = suf + 256;
+  if (cand >= 0 && cand == best) *above_s = cand_above;
+  __syncthreads();
   if (tid == 0) {
     PeState s = *stp;
     int cut = best;
@@ -316,8 +322,8 @@ __device__ void pe_find(const crisp_params& p, PeState* stp, uint32_t* gc, doubl
     if (cut < 0) {
       s.all = 1;                       // the whole triangle sums below gamma
     } else {
-      double above = above0;
-      for (int bk = nbk - 1; bk > cut; --bk) above += __ldcg(gs + bk);
+      // every bucket above the lowest non-empty one: the scan total without it
+      const double above = cut == best ? *above_s : above0 + suf[255] - __ldcg(gs + cut);
       s.prefix |= uint32_t(cut) << shift;
       s.above_sum = above;
       if (level == 2) {
