@@ -124,6 +124,15 @@ def launches_per_step(router: str) -> dict:
     return {"route": route, "select": select, "attention": 1, "total": route + select + 1}
 
 
+def workload_config(w, args) -> dict:
+    """The config block both arms report for a workload and its hyper-parameters."""
+    return {"workload": w.name, "batch": w.batch, "h_q": w.h_q, "h_kv": w.h_kv,
+            "head_dim": w.head_dim, "seq_len": w.seqlen, "block": w.block,
+            "diffuse_frac": w.diffuse_frac, "alpha": args.alpha, "gamma": args.gamma,
+            "router": args.router, "vs_rule": args.vs_rule, "granularity": args.granularity,
+            **({"lengths": list(w.lengths)} if w.lengths is not None else {})}
+
+
 def executed_flops(tile_cnt_sum: int, block: int, d: int) -> float:
     """4 * B^2 * d per executed tile (QK^T and PV); diagonal tiles count in full."""
     return float(tile_cnt_sum) * 4.0 * block * block * d
@@ -257,12 +266,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": round(ms, 3), "unit": "ms", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": False,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "batch": w.batch, "h_q": w.h_q, "h_kv": w.h_kv,
-                   "head_dim": w.head_dim, "seq_len": w.seqlen, "block": w.block,
-                   "diffuse_frac": w.diffuse_frac, "alpha": args.alpha, "gamma": args.gamma,
-                   "router": args.router, "vs_rule": args.vs_rule, "granularity": args.granularity,
-                   "parallelism": f"replicas{world}",
-                   **({"lengths": list(w.lengths)} if w.lengths is not None else {}),
+        "config": {**workload_config(w, args), "parallelism": f"replicas{world}",
                    "l2": "flushed between steps" if flush is not None else
                          f"inputs ({in_bytes / 2**30:.1f} GiB) larger than L2"},
         "stages_ms": {k_: round(v_, 3) for k_, v_ in stages.items()},
@@ -418,8 +422,8 @@ def oracle_sample(w, args, inp, budget_s: float):
         tiles[h] = int(r["mask"].sum())
         rng = np.random.default_rng(h)
         for qb in sorted(set([nb - 1] + [int(x) for x in rng.integers(0, nb, size=3)])):
-            if time.perf_counter() - t_start > budget_s:
-                break
+            if attn_ms_per_tile and time.perf_counter() - t_start > budget_s:
+                break                                      # at least one query block is always timed
             t0 = time.perf_counter()
             O.masked_attention_rows(qh, kh, vh, r["mask"], w.block, prm.scale(w.head_dim), [qb],
                                     r.get("vs_tokens"))
@@ -455,8 +459,7 @@ def run_reference(args):
             "warmup": args.warmup, "ms_per_step": round(v, 1), "higher_is_better": False,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": w.name, "seq_len": w.seqlen, "h_q": w.h_q, "h_kv": w.h_kv,
-                       "head_dim": w.head_dim, "block": w.block, "alpha": args.alpha},
+            "config": {**workload_config(w, args), "parallelism": "host cores"},
             "cpu_baseline": {"value": round(v, 1), "unit": "ms", "cores": threads, "kind": "oracle",
                              "sample": desc + " (extrapolated)"},
             "e2e": {"value": round(v, 1), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
