@@ -118,6 +118,13 @@ def test_variable_length_batch(kw):
     _check(Workload(**base))
 
 
+@pytest.mark.parametrize("router,vs_rule", [("jsd", "gamma"), ("cstruct", "alpha_median")])
+def test_variable_length_batch_routers_and_rules(router, vs_rule):
+    w = Workload("varlen_r", 3, 4, 2, 128, 2048 + 64, 128, n_vertical=2, diffuse_frac=0.5, sink_logit=8.0,
+                 lengths=(2048 + 64, 1111, 3 * 128 + 5))
+    _check(w, router=router, vs_rule=vs_rule)
+
+
 def test_variable_length_dense_equals_oracle():
     w = Workload("varlen_dense", 2, 2, 1, 128, 1536, 128, lengths=(1536 - 100, 700))
     q, k, v, _ = make_qkv(w)
