@@ -252,8 +252,11 @@ def run_ours(args, rank, world, local_rank):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         e2e_ms = max_over_ranks([e0.elapsed_time(e1) / args.steps], dev)[0]
-        e2e = {"value": round(e2e_ms, 3), "unit": "ms",
-               "h2d_bytes_per_step": int(in_bytes), "d2h_bytes_per_step": int(o.numel() * o.element_size()),
+        # bytes that cross PCIe: with lengths, only each sequence's own rows
+        rows = sum(w.length(b) for b in range(w.batch))
+        h2d = rows * (w.h_q + 2 * w.h_kv) * w.head_dim * q.element_size()
+        d2h = rows * w.h_q * w.head_dim * o.element_size()
+        e2e = {"value": round(e2e_ms, 3), "unit": "ms", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "path": "prefill_from_host (pinned host Q/K/V in, O out; copies overlapped per KV head)"}
         del hq, hk, hv, ho
 

@@ -10,6 +10,10 @@ chunks. Every compute step is a call through the C ABI (crisp_route,
 crisp_select, crisp_sparse_prefill); this module only moves memory and
 orders streams.
 
+With per-sequence lengths only the rows a sequence holds cross PCIe (one
+copy per head); rows of o (and lse) past a sequence's length are left as
+they were on the host.
+
 The call is asynchronous with respect to the host and ordered on the
 caller's current stream: the pipeline starts after the work already queued
 there and the current stream waits for its last copy.
@@ -68,9 +72,11 @@ def prefill_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torc
             ws = torch.empty(B.crisp_workspace_size(p), dtype=torch.uint8, device=dev)
             ws[:256].zero_()
             slots.append({
+                # rows past a sequence keep older (finite) contents; v starts at
+                # zero because those rows of its last tile meet exact-zero weights
                 "q": torch.empty((1, cq, n, d), dtype=q.dtype, device=dev),
                 "k": torch.empty((1, ck, n, d), dtype=k.dtype, device=dev),
-                "v": torch.empty((1, ck, n, d), dtype=v.dtype, device=dev),
+                "v": torch.zeros((1, ck, n, d), dtype=v.dtype, device=dev),
                 "o": torch.empty((1, cq, n, d), dtype=q.dtype, device=dev),
                 "lse": torch.empty((1, cq, n), dtype=torch.float32, device=dev) if lse is not None else None,
                 "ws": ws,
@@ -94,10 +100,18 @@ def prefill_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torc
         # inputs of this slot are free once the compute of its previous chunk ended
         if sl["used"]:
             s_in.wait_event(sl["cmp"])
+        nv = n if seq_lens is None else int(seq_lens[b])
         with torch.cuda.stream(s_in):
-            sl["q"][0].copy_(q[b, qs], non_blocking=True)
-            sl["k"][0].copy_(k[b, ks], non_blocking=True)
-            sl["v"][0].copy_(v[b, ks], non_blocking=True)
+            if nv == n:
+                sl["q"][0].copy_(q[b, qs], non_blocking=True)
+                sl["k"][0].copy_(k[b, ks], non_blocking=True)
+                sl["v"][0].copy_(v[b, ks], non_blocking=True)
+            else:                                            # the sequence's rows only, per head
+                for i in range(cq):
+                    sl["q"][0, i, :nv].copy_(q[b, qs.start + i, :nv], non_blocking=True)
+                for i in range(ck):
+                    sl["k"][0, i, :nv].copy_(k[b, ks.start + i, :nv], non_blocking=True)
+                    sl["v"][0, i, :nv].copy_(v[b, ks.start + i, :nv], non_blocking=True)
         sl["in"].record(s_in)
         # outputs of this slot are free once its previous copy out ended
         s_cmp.wait_event(sl["in"])
@@ -116,9 +130,15 @@ def prefill_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torc
         sl["cmp"].record(s_cmp)
         s_out.wait_event(sl["cmp"])
         with torch.cuda.stream(s_out):
-            o[b, qs].copy_(sl["o"][0], non_blocking=True)
-            if lse is not None:
-                lse[b, qs].copy_(sl["lse"][0], non_blocking=True)
+            if nv == n:
+                o[b, qs].copy_(sl["o"][0], non_blocking=True)
+                if lse is not None:
+                    lse[b, qs].copy_(sl["lse"][0], non_blocking=True)
+            else:
+                for i in range(cq):
+                    o[b, qs.start + i, :nv].copy_(sl["o"][0, i, :nv], non_blocking=True)
+                    if lse is not None:
+                        lse[b, qs.start + i, :nv].copy_(sl["lse"][0, i, :nv], non_blocking=True)
         sl["out"].record(s_out)
         sl["used"] = True
     # the caller's stream continues after the last copy out and the last compute

@@ -42,11 +42,10 @@ def test_pipeline_matches_device_path(kv_per_chunk):
     assert torch.equal(out["pattern"].cpu(), pattern.cpu())
     assert int(out["tile_cnt_sum"]) == int(tcnt.sum())
     o_ref, lse_ref = o_ref.cpu(), lse_ref.cpu()
-    err = (ho.float() - o_ref.float()).abs()
-    assert float(err.max()) <= 2e-2 and float(err.mean()) <= 2e-3
-    same = torch.isfinite(lse_ref)
-    assert torch.allclose(hl[same], lse_ref[same], atol=2e-3, rtol=0)
-    assert torch.equal(hl[~same], lse_ref[~same])      # padding rows: -inf on both paths
+    for b, n in enumerate(w.lengths):                  # only a sequence's own rows are copied back
+        err = (ho[b, :, :n].float() - o_ref[b, :, :n].float()).abs()
+        assert float(err.max()) <= 2e-2 and float(err.mean()) <= 2e-3
+        assert torch.allclose(hl[b, :, :n], lse_ref[b, :, :n], atol=2e-3, rtol=0)
 
 
 def test_pipeline_rejects_pageable_inputs():
