@@ -27,7 +27,7 @@ PATTERN_VS, PATTERN_PE = 0, 1
 
 EXPORTED = ("crisp_version", "crisp_status_string", "crisp_check_params", "crisp_workspace_size",
             "crisp_route", "crisp_select", "crisp_sparse_prefill", "crisp_dense_prefill",
-            "crisp_get_device_status", "crisp_route_noalloc")
+            "crisp_get_device_status", "crisp_route_noalloc", "crisp_selftest_wait_timeout")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -106,6 +106,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.crisp_dense_prefill.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.crisp_route_noalloc.restype = i32
     lib.crisp_route_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
+    lib.crisp_selftest_wait_timeout.restype = i32
+    lib.crisp_selftest_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
     lib.crisp_get_device_status.restype = i32
     lib.crisp_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), vp]
     _lib = lib
@@ -248,3 +250,11 @@ def crisp_prefill(q, k, v, ws=None, want_mask=False, stream=None, **kw):
     o, lse = crisp_sparse_prefill(p, q, k, v, tile_idx, tile_cnt, ws, stream=stream)
     return {"o": o, "lse": lse, "pattern": pattern, "score": score, "p_v": p_v, "p_s": p_s,
             "mask": mask, "tile_idx": tile_idx, "tile_cnt": tile_cnt, "params": p, "ws": ws}
+
+
+def crisp_selftest_wait_timeout(ws: torch.Tensor, limit_cycles: int = 1 << 20, stream=None) -> None:
+    """Runs the bounded-wait self-test on ws's device (see include/crisp.h):
+    afterwards crisp_get_device_status(ws) reports CRISP_ERR_TIMEOUT (-5)."""
+    _need_cuda(ws)
+    _check("crisp_selftest_wait_timeout", load_library().crisp_selftest_wait_timeout(
+        _ptr(ws), int(limit_cycles), _stream(stream)))

@@ -187,6 +187,15 @@ int crisp_dense_prefill(const crisp_params* p, const void* q, const void* k, con
 int crisp_route_noalloc(const crisp_params* p, const void* q, const void* k, int32_t* pattern,
                         float* score, float* p_v, float* p_s, void* stream);
 
+/* Diagnostic: exercises the bounded wait that every pipelined kernel of the
+ * library uses (on an mbarrier phase, a TMA copy or a tensor-core commit).
+ * One CTA waits on an mbarrier nothing arrives on, gives up after
+ * `limit_cycles` (1 .. 2^31) SM clock cycles, records CRISP_ERR_TIMEOUT in
+ * the status word of `ws` (256-byte aligned, at least 256 bytes; read it with
+ * crisp_get_device_status) and returns; the context stays usable. Returns
+ * CRISP_ERR_ARG for a bad workspace or limit. The paper has no counterpart. */
+int crisp_selftest_wait_timeout(void* ws, long long limit_cycles, void* stream);
+
 /* Synchronises `stream`, copies the device status word out of `ws` into
  * *status (CRISP_OK or CRISP_ERR_TIMEOUT / CRISP_ERR_DEVICE) and clears it.
  * Returns CRISP_OK unless the copy itself failed. */

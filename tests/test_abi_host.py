@@ -95,6 +95,14 @@ def test_entry_points_validate_before_launch(lib):
     assert lib.crisp_get_device_status(None, ctypes.byref(st), None) == -1
 
 
+def test_selftest_validates_before_launch(lib):
+    fake = ctypes.c_void_p(1 << 20)                       # aligned, never dereferenced on failure
+    assert lib.crisp_selftest_wait_timeout(None, 1000, None) == -1
+    assert lib.crisp_selftest_wait_timeout(ctypes.c_void_p((1 << 20) + 8), 1000, None) == -1
+    assert lib.crisp_selftest_wait_timeout(fake, 0, None) == -1
+    assert lib.crisp_selftest_wait_timeout(fake, (1 << 31) + 1, None) == -1
+
+
 def test_params_struct_layout_matches_header(lib, tmp_path):
     # 10 int32 + 4 float fields, then the 8-byte seq_lens pointer; the C
     # compiler's view of include/crisp.h must agree with the ctypes mirror
