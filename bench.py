@@ -448,6 +448,19 @@ def oracle_sample(w, args, inp, budget_s: float):
     return ms, desc, threads
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), or the platform's."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
 def run_reference(args):
     from synthetic import WORKLOADS
     w = WORKLOADS[args.workload].with_(seed=args.seed)
@@ -464,7 +477,7 @@ def run_reference(args):
             "impl": "reference",
             "config": {**workload_config(w, args), "parallelism": "host cores"},
             "cpu_baseline": {"value": round(v, 1), "unit": "ms", "cores": threads, "kind": "oracle",
-                             "sample": desc + " (extrapolated)"},
+                             "cpu": cpu_model(), "sample": desc + " (extrapolated)"},
             "e2e": {"value": round(v, 1), "unit": "ms", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -517,7 +530,7 @@ def main():
         if w.batch == 1:
             ms, desc, threads = oracle_sample(w, args, oracle_inputs(w), budget_s=args.cpu_budget)
             line["cpu_baseline"] = {"value": round(ms, 1), "unit": "ms", "cores": threads, "kind": "oracle",
-                                    "sample": desc + " (extrapolated)"}
+                                    "cpu": cpu_model(), "sample": desc + " (extrapolated)"}
         else:   # the sampler extrapolates one sequence's heads; batches are not sampled
             line["cpu_baseline"] = None
             line["cpu_baseline_note"] = "oracle sample covers single-sequence workloads only"

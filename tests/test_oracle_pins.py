@@ -403,6 +403,21 @@ def test_ragged_block_scores_bruteforce():
         assert abs(c - (first + last)) < 1e-13
 
 
+def test_ragged_pooled_estimate_bruteforce():
+    # Algorithm 5 line 3 on a partial last block: the block means of K run over
+    # the keys each block holds; the estimate is a softmax over all N_b blocks
+    rng = _rng(27)
+    B, n, d = 8, 8 * 5 + 3, 4
+    q_hat, k = rng.standard_normal((B, d)), rng.standard_normal((n, d))
+    qm = [sum(q_hat[r][c] for r in range(B)) / B for c in range(d)]
+    blocks = [list(range(i, min(i + B, n))) for i in range(0, n, B)]
+    kbar = [[sum(k[j][c] for j in blk) / len(blk) for c in range(d)] for blk in blocks]
+    z = [0.6 * sum(qm[c] * kb[c] for c in range(d)) for kb in kbar]
+    e = [math.exp(x - max(z)) for x in z]
+    want = [x / sum(e) for x in e]
+    np.testing.assert_allclose(O.pooled_estimate_last_block(q_hat, k, B, 0.6), want, atol=1e-14)
+
+
 def test_ragged_pooling_means_partial_block():
     x = np.arange(22, dtype=np.float64).reshape(11, 2)        # 11 rows, B = 4: 4 + 4 + 3
     pooled = O.pe_pool(x, 4)
