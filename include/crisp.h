@@ -17,12 +17,13 @@
  *    Every pointer must be 16-byte aligned.
  *  - The caller owns all memory, including the workspace `ws` of
  *    `ws_bytes` >= crisp_workspace_size(p) bytes (256-byte aligned). The
- *    library allocates no device memory and keeps no global state.
+ *    library allocates no device memory and keeps no global state, except
+ *    the fixed scratch array of crisp_route_noalloc (see there).
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
  *    default stream). The return value covers argument validation and
  *    launch errors only; kernel-side errors (a bounded wait that ran out,
- *    an out-of-range tile index) are recorded in a status word held in the
- *    first 8 bytes of `ws`, read back (and cleared) with
+ *    an out-of-range tile index or sequence length) are recorded in a status
+ *    word held in the first 8 bytes of `ws`, read back (and cleared) with
  *    crisp_get_device_status(). crisp_route and crisp_dense_prefill start a
  *    prefill and clear the word (crisp_route also clears the per-head
  *    completion counters its kernels keep right after it); a caller who runs
