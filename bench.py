@@ -133,6 +133,27 @@ def workload_config(w, args) -> dict:
             **({"lengths": list(w.lengths)} if w.lengths is not None else {})}
 
 
+def stage_algorithmic_bytes(w, pattern) -> dict:
+    """HBM bytes the routing and selection stages must move at least once
+    (algorithmic, not measured): routing reads K once per KV head (the proxy
+    is bound by its exp2 work, so this only says how far from HBM-bound it
+    is); selection pools K of the KV heads with a PE query head and Q of the
+    PE heads, then passes over each PE head's N_b(N_b+1)/2 estimate entries
+    (fp32) seven times: written by the logits, read and written by the
+    normalisation, read by three radix levels, the tie count and the tile
+    builder."""
+    g = w.h_q // w.h_kv
+    d2 = w.head_dim * 2
+    route = sum(w.length(b) * w.h_kv * d2 for b in range(w.batch))
+    select = 0
+    for b in range(w.batch):
+        n = w.length(b)
+        nb = -(-n // w.block)
+        pe = [h for h in range(w.h_q) if pattern[b * w.h_q + h] == 1]
+        select += (len(pe) + len({h // g for h in pe})) * n * d2 + len(pe) * nb * (nb + 1) // 2 * 4 * 7
+    return {"route": route, "select": select}
+
+
 def executed_flops(tile_cnt_sum: int, block: int, d: int) -> float:
     """4 * B^2 * d per executed tile (QK^T and PV); diagonal tiles count in full."""
     return float(tile_cnt_sum) * 4.0 * block * block * d
@@ -183,6 +204,7 @@ def run_ours(args, rank, world, local_rank):
     n_vs = int((pattern == 0).sum().item())
     nbv = [-(-w.length(b) // w.block) for b in range(w.batch)]        # each sequence's blocks
     causal_tiles = p.h_q * sum(x * (x + 1) // 2 for x in nbv)
+    stage_bytes = stage_algorithmic_bytes(w, pattern.cpu().tolist())
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     if world > 1:
@@ -282,9 +304,15 @@ def run_ours(args, rank, world, local_rank):
         "attend_tflops": round(attn_tflops, 1), "dense_tflops": round(dense_tflops, 1),
         "roofline": {"bound": "tensor", "kernel": "attention (sparse)", "achieved": round(attn_tflops, 1),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(attn_tflops / peak, 4),
+                     "frac_of_burst": round(attn_tflops / peaks["bf16_tflops"], 4),
+                     "frac_of_spec_2250": round(attn_tflops / 2250.0, 4),
                      "peak_source": f"{peaks['source']} bf16 "
                                     f"{'sustained' if peak == peaks['bf16_tflops_sustained'] else 'burst'}",
                      "traffic": None},
+        "stage_hbm": {k_: {"algorithmic_bytes": int(v_),
+                           "achieved_gbs": round(v_ / (stages[k_] * 1e-3) / 1e9, 1),
+                           "frac_of_hbm": round(v_ / (stages[k_] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+                      for k_, v_ in stage_bytes.items()},
         "e2e": e2e,
         "gpu_launches": launches_per_step(args.router)["total"] * args.steps,
         "device_status": status,
