@@ -120,3 +120,13 @@ def test_params_struct_layout_matches_header(lib, tmp_path):
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
     assert [int(x) for x in out] == [ctypes.sizeof(B.CrispParams), B.CrispParams.seq_lens.offset,
                                      B.CrispParams.sm_scale.offset, B.CrispParams.vs_granularity.offset]
+
+
+def test_binding_rejects_host_lengths_and_bad_enums():
+    import torch
+    with pytest.raises(ValueError):
+        B.make_params(2, 4, 2, 4096, 128, seq_lens=torch.tensor([4096, 100], dtype=torch.int32))
+    with pytest.raises(KeyError):
+        B.make_params(1, 4, 2, 4096, 128, vs_rule="median")
+    p = B.make_params(1, 4, 2, 4096, 128, granularity="token", vs_rule="alpha_median", router="jsd")
+    assert (p.vs_granularity, p.vs_rule, p.router) == (1, 2, 1)
