@@ -473,12 +473,15 @@ __global__ void __launch_bounds__(256) pe_eqcount_kernel(crisp_params p, const i
 }
 
 // ---------------------------------------------------------------------------
-// Tile lists: one warp per (head, query block). Lanes cover 4 consecutive
-// key blocks per step (uchar4 mask stores), a warp scan compacts the active
-// ids in ascending order.
-// VS: tile active iff kb in S_v u {0}, or qb-kb or qb-kb-1 in the offset set
-//     O = {N_b-1-j : j in S_s} u {0}.
-// PE: active iff chosen by the gamma cut, or kb == qb, or kb == 0.
+// Tile lists: one warp per (head, query block); a warp scan compacts the
+// active ids in ascending order.
+// VS: tile active iff kb in S_v u {0}, or a selected slash block (or N_b-1)
+//     meets the tile: for a sequence whose length is a multiple of B, qb-kb
+//     or qb-kb-1 in the offset set O = {N_b-1-j : j in S_s} u {0}; for a
+//     partial last block see the rule below. Lanes take 32 key blocks each
+//     from the selection bitmasks.
+// PE: active iff chosen by the gamma cut, or kb == qb, or kb == 0; lanes take
+//     4 consecutive key blocks per step.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) build_tiles_kernel(crisp_params p, const int32_t* pattern,
                                                           void* ws, uint8_t* __restrict__ mask,
