@@ -588,6 +588,27 @@ def test_planted_recovery_tiny_workload():
     assert w.n_blocks - 1 in h0["s_s"]          # local diagonal block
     assert h0["c_struct"] > 0.5 > 0.2 > h1["c_struct"]
     assert h0["mask"].sum() < h1["mask"].sum()
+    # Appendix F: a diffuse (PE) head does not reach gamma within its top 50 blocks
+    assert len(h1["pe_selected"]) > 50
+
+
+def test_alpha_rule_is_sink_aware():
+    # Section 4.3: the floor excludes the anchors, so it falls as the sink grows;
+    # moving mass from the middle blocks into the sink (scaling them all by c)
+    # lowers mu by the same factor and leaves the selected middle blocks unchanged
+    rng = _rng(28)
+    nb = 24
+    p = rng.dirichlet(np.full(nb, 0.4))
+    base = O.vs_index_alpha(p, 1.0, 2)
+    mu = float(O.noise_floor(p))
+    for c in (0.8, 0.5, 0.2):
+        q = p.copy()
+        q[1:-1] *= c
+        q[0] += (1 - c) * p[1:-1].sum()
+        assert float(O.noise_floor(q)) < mu
+        assert abs(float(O.noise_floor(q)) - c * mu) < 1e-6 * mu
+        got = O.vs_index_alpha(q, 1.0, 2)
+        assert set(got.tolist()) - {0} == set(base.tolist()) - {0}, c
 
 
 def test_planted_recovery_verticals_and_jsd_agreement():
