@@ -5,8 +5,9 @@
 // that the tile lists select (the union over the query blocks the tile covers,
 // with a per-block membership mask), in ascending order: steps j = 0..n-1.
 //
-//   warp 8 (one lane)  TMA producer of Q and of the K tiles (two-slot ring).
-//   warp 10 (one lane) TMA producer of the V tiles (two-slot ring).
+//   warp 8 (one lane)  TMA producer of Q and of the K tiles (a ring of 2
+//                      slots for d = 128, 4 for d = 64).
+//   warp 10 (one lane) TMA producer of the V tiles (a ring of the same depth).
 //   warp 9 (one lane)  UMMA issuer of S_j = Q K_j^T into TMEM buffer j%2, as
 //                      soon as the softmax has read S_{j-2} from that buffer.
 //   warp 11 (one lane) UMMA issuer of O_{j%2} += P_j V_j into one of two TMEM
