@@ -93,8 +93,8 @@ def prefill_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torc
         pattern_all = torch.empty(bsz * hq, dtype=torch.int32, device=dev)
         tiles = torch.zeros((), dtype=torch.int64, device=dev)
     chunks = [(b, h0) for b in range(bsz) for h0 in range(0, hkv, ck)]
-    for i, (b, h0) in enumerate(chunks):
-        sl = slots[i % 2]
+    for ci, (b, h0) in enumerate(chunks):
+        sl = slots[ci % 2]
         qs = slice(h0 * g, h0 * g + cq)
         ks = slice(h0, h0 + ck)
         # inputs of this slot are free once the compute of its previous chunk ended
@@ -107,11 +107,11 @@ def prefill_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torc
                 sl["k"][0].copy_(k[b, ks], non_blocking=True)
                 sl["v"][0].copy_(v[b, ks], non_blocking=True)
             else:                                            # the sequence's rows only, per head
-                for i in range(cq):
-                    sl["q"][0, i, :nv].copy_(q[b, qs.start + i, :nv], non_blocking=True)
-                for i in range(ck):
-                    sl["k"][0, i, :nv].copy_(k[b, ks.start + i, :nv], non_blocking=True)
-                    sl["v"][0, i, :nv].copy_(v[b, ks.start + i, :nv], non_blocking=True)
+                for hh in range(cq):
+                    sl["q"][0, hh, :nv].copy_(q[b, qs.start + hh, :nv], non_blocking=True)
+                for hh in range(ck):
+                    sl["k"][0, hh, :nv].copy_(k[b, ks.start + hh, :nv], non_blocking=True)
+                    sl["v"][0, hh, :nv].copy_(v[b, ks.start + hh, :nv], non_blocking=True)
         sl["in"].record(s_in)
         # outputs of this slot are free once its previous copy out ended
         s_cmp.wait_event(sl["in"])
@@ -135,10 +135,10 @@ def prefill_from_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torc
                 if lse is not None:
                     lse[b, qs].copy_(sl["lse"][0], non_blocking=True)
             else:
-                for i in range(cq):
-                    o[b, qs.start + i, :nv].copy_(sl["o"][0, i, :nv], non_blocking=True)
+                for hh in range(cq):
+                    o[b, qs.start + hh, :nv].copy_(sl["o"][0, hh, :nv], non_blocking=True)
                     if lse is not None:
-                        lse[b, qs.start + i, :nv].copy_(sl["lse"][0, i, :nv], non_blocking=True)
+                        lse[b, qs.start + hh, :nv].copy_(sl["lse"][0, hh, :nv], non_blocking=True)
         sl["out"].record(s_out)
         sl["used"] = True
     # the caller's stream continues after the last copy out and the last compute
