@@ -7,8 +7,7 @@ GPU's own tile mask: max-abs <= 2e-2 and mean-abs <= 2e-3.
 """
 from __future__ import annotations
 
-import math
-from typing import Dict, Optional, Sequence
+from typing import Sequence
 
 import numpy as np
 import torch

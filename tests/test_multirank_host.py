@@ -3,8 +3,6 @@ the max over ranks of each rank's own CUDA-event time."""
 import os
 import socket
 
-import pytest
-import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
