@@ -130,3 +130,44 @@ def test_binding_rejects_host_lengths_and_bad_enums():
         B.make_params(1, 4, 2, 4096, 128, vs_rule="median")
     p = B.make_params(1, 4, 2, 4096, 128, granularity="token", vs_rule="alpha_median", router="jsd")
     assert (p.vs_granularity, p.vs_rule, p.router) == (1, 2, 1)
+
+
+def test_c_program_links_and_calls_the_library(lib, tmp_path):
+    # a plain C99 program, linked against libcrisp.so, makes the host-side
+    # calls of the C example (no device work): version, validation, workspace
+    # size, status strings, and an entry point refusing NULL pointers
+    src = tmp_path / "use.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "crisp.h"
+int main(void) {
+  crisp_params p = {.batch = 1, .h_q = 32, .h_kv = 8, .seqlen = 524288, .head_dim = 128,
+                    .block = 128, .alpha = 1.0f, .gamma = 0.95f, .tau_proxy = 0.2f,
+                    .tau_jsd = 0.1f, .k_min_blocks = 8, .router = CRISP_ROUTER_CSTRUCT,
+                    .vs_rule = CRISP_VS_ALPHA, .sm_scale = 0.0f,
+                    .vs_granularity = CRISP_GRAN_TILE, .seq_lens = NULL};
+  int ok = crisp_check_params(&p);
+  size_t ws = crisp_workspace_size(&p);
+  int route = crisp_route(&p, NULL, NULL, NULL, ws, NULL, NULL, NULL, NULL, NULL);
+  p.seqlen = 2 * 128;                      /* N_b = 2: below the minimum of 3 blocks */
+  printf("%d %d %zu %d %d %zu|%s|%s\n", crisp_version(), ok, ws, route, crisp_check_params(&p),
+         crisp_workspace_size(&p), crisp_status_string(CRISP_OK), crisp_status_string(CRISP_ERR_SHAPE));
+  return 0;
+}
+''')
+    exe = tmp_path / "use"
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.join(root, "dynamic_block_sparse_qk_b200")
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(root, "include"), str(src), "-o", str(exe),
+                    "-L", pkg, "-lcrisp", "-Wl,-rpath," + pkg], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.strip()
+    nums, ok_name, shape_name = out.split("|")
+    version, ok, ws, route, bad, ws_bad = (int(x) for x in nums.split())
+    p = B.make_params(1, 32, 8, 524288, 128)
+    assert version == lib.crisp_version()
+    assert ok == 0 and ws == B.crisp_workspace_size(p) > 0
+    assert route == -1                                     # CRISP_ERR_ARG, nothing launched
+    assert bad == -2 and ws_bad == 0                       # CRISP_ERR_SHAPE
+    lib.crisp_status_string.restype = ctypes.c_char_p
+    assert ok_name == lib.crisp_status_string(0).decode()
+    assert shape_name == lib.crisp_status_string(-2).decode()
