@@ -171,3 +171,14 @@ int main(void) {
     lib.crisp_status_string.restype = ctypes.c_char_p
     assert ok_name == lib.crisp_status_string(0).decode()
     assert shape_name == lib.crisp_status_string(-2).decode()
+
+
+def test_host_input_prefill_rejects_unpinned_tensors():
+    # prefill_from_host copies asynchronously from page-locked memory only; a
+    # pageable (or device) tensor is refused before any stream or copy exists
+    import torch
+    from dynamic_block_sparse_qk_b200 import prefill_from_host
+    q = torch.zeros(1, 4, 1024, 64, dtype=torch.bfloat16)
+    k = torch.zeros(1, 2, 1024, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="pinned host memory"):
+        prefill_from_host(q, k, k.clone(), torch.empty_like(q), block=64)
