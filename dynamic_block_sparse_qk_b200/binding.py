@@ -27,7 +27,8 @@ PATTERN_VS, PATTERN_PE = 0, 1
 
 EXPORTED = ("crisp_version", "crisp_status_string", "crisp_check_params", "crisp_workspace_size",
             "crisp_route", "crisp_select", "crisp_sparse_prefill", "crisp_dense_prefill",
-            "crisp_get_device_status", "crisp_route_noalloc", "crisp_selftest_wait_timeout")
+            "crisp_get_device_status", "crisp_route_noalloc", "crisp_selftest_wait_timeout",
+            "crisp_selftest_pipeline_timeout")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -108,6 +109,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.crisp_route_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
     lib.crisp_selftest_wait_timeout.restype = i32
     lib.crisp_selftest_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
+    lib.crisp_selftest_pipeline_timeout.restype = i32
+    lib.crisp_selftest_pipeline_timeout.argtypes = [P, vp, vp, vp, vp, vp, sz, ctypes.c_longlong, vp]
     lib.crisp_get_device_status.restype = i32
     lib.crisp_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), vp]
     _lib = lib
@@ -231,6 +234,8 @@ def crisp_route_noalloc(p: CrispParams, q, k, pattern=None, score=None, p_v=None
 
 
 def crisp_get_device_status(ws, stream=None) -> int:
+    """Reads and clears the device status word of a workspace (ws = None:
+    the scratch array of crisp_route_noalloc on the current device)."""
     st = ctypes.c_int32(0)
     _check("crisp_get_device_status",
            load_library().crisp_get_device_status(_ptr(ws), ctypes.byref(st), _stream(stream)))
@@ -258,3 +263,14 @@ def crisp_selftest_wait_timeout(ws: torch.Tensor, limit_cycles: int = 1 << 20, s
     _need_cuda(ws)
     _check("crisp_selftest_wait_timeout", load_library().crisp_selftest_wait_timeout(
         _ptr(ws), int(limit_cycles), _stream(stream)))
+
+
+def crisp_selftest_pipeline_timeout(p: CrispParams, q, k, v, o, ws, limit_cycles: int = 64,
+                                    stream=None) -> None:
+    """Runs the proxy and attention kernels with every pipeline wait cut to
+    ``limit_cycles`` (see include/crisp.h): afterwards
+    crisp_get_device_status(ws) reports CRISP_ERR_TIMEOUT (-5)."""
+    _need_cuda(q, k, v, o, ws)
+    _check("crisp_selftest_pipeline_timeout", load_library().crisp_selftest_pipeline_timeout(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ws), ws.numel(), int(limit_cycles),
+        _stream(stream)))

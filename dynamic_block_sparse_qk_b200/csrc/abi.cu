@@ -138,9 +138,32 @@ int crisp_dense_prefill(const crisp_params* p, const void* q, const void* k, con
   return to_status(e);
 }
 
-int crisp_get_device_status(void* ws, int32_t* status, void* stream) {
-  if (!ws || !status || !aligned(ws, 256)) return CRISP_ERR_ARG;
+int crisp_selftest_pipeline_timeout(const crisp_params* p, const void* q, const void* k, const void* v,
+                                    void* o, void* ws, size_t ws_bytes, long long limit_cycles,
+                                    void* stream) {
+  int s = check_params(p);
+  if (s) return s;
+  if ((s = check_ws(p, ws, ws_bytes))) return s;
+  if (!q || !k || !v || !o) return CRISP_ERR_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16)) return CRISP_ERR_ARG;
+  if (limit_cycles < 1 || limit_cycles >= (1ll << 20)) return CRISP_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the proxy statistics kernel of crisp_route, then the attention kernel of
+  // crisp_dense_prefill, both with every pipeline wait cut to limit_cycles
+  cudaError_t e = cudaMemsetAsync(ws, 0, route_clear_bytes(*p), st);
+  if (e == cudaSuccess) e = run_proxy_stats(*p, q, k, ws, st, limit_cycles);
+  if (e == cudaSuccess) e = run_attention(*p, q, k, v, nullptr, nullptr, o, nullptr, ws, st, limit_cycles);
+  return to_status(e);
+}
+
+int crisp_get_device_status(void* ws, int32_t* status, void* stream) {
+  if (!status) return CRISP_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!ws) {                 // the scratch array of crisp_route_noalloc on this device
+    const int a = noalloc_scratch(&ws, st);
+    if (a != CRISP_OK) return a;
+  }
+  if (!aligned(ws, 256)) return CRISP_ERR_ARG;
   int32_t word = 0;
   cudaError_t e = cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);

@@ -29,8 +29,9 @@
 //
 // Every mbarrier wait is bounded; a wait that runs out records
 // CRISP_ERR_TIMEOUT in the workspace status word and raises a CTA abort flag,
-// after which all roles leave their loops, the producer waits (bounded) for
-// its copies in flight and the TMEM allocation is released.
+// after which all roles leave their loops, the producers wait (bounded) for
+// their copies in flight, each UMMA issuer waits (bounded) for a final commit
+// of everything it issued, and only then is the TMEM allocation released.
 #include <climits>
 
 #include "common.cuh"
@@ -61,7 +62,8 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_VRING + NSLOT * T_BYTES;
   static constexpr int B_Q = 0, B_KFULL = 1, B_KEMPTY = 1 + NSLOT, B_VFULL = 1 + 2 * NSLOT,
                        B_VEMPTY = 1 + 3 * NSLOT, B_S = 1 + 4 * NSLOT, B_SFREE = B_S + 2,
-                       B_P = B_SFREE + 2, B_PV = B_P + 2, B_O = B_PV + 2, N_BARS = B_O + 1;
+                       B_P = B_SFREE + 2, B_PV = B_P + 2, B_O = B_PV + 2, B_SDRAIN = B_O + 1,
+                       N_BARS = B_SDRAIN + 1;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * N_BARS;
   static constexpr int OFF_ABORT = OFF_TMEM + 8;
   static constexpr int SMEM = OFF_ABORT + 8 + 1024;   // + alignment slack
@@ -177,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                    const __grid_constant__ CUtensorMap tmv, const int32_t* __restrict__ tile_idx,
                    const int32_t* __restrict__ tile_cnt, __nv_bfloat16* __restrict__ o,
-                   float* __restrict__ lse, crisp_params p, void* ws) {
+                   float* __restrict__ lse, crisp_params p, void* ws, long long wait_limit) {
   using C = Cfg<D>;
   constexpr int NSLOT = C::NSLOT;
   extern __shared__ unsigned char smem_raw[];
@@ -234,6 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(BAR(C::B_PV + g), 1);
     }
     mbar_init(BAR(C::B_O), 1);
+    mbar_init(BAR(C::B_SDRAIN), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -269,19 +272,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t bits;
       while (it.next(kt, bits)) {
         const int s = t % NSLOT, u = t / NSLOT;
-        if (u >= 1 && !mbar_wait(BAR(bempty + s), (u - 1) & 1, abort_flag, status, 1)) break;
+        if (u >= 1 && !mbar_wait(BAR(bempty + s), (u - 1) & 1, abort_flag, status, 1, wait_limit)) break;
         mbar_arrive_expect_tx(BAR(bfull + s), C::T_BYTES);
         for (int box = 0; box < D / 64; ++box)
           tma_load_2d(ring + s * C::T_BYTES + box * BN * 128, map, box * 64, kv_row0 + kt * BN, BAR(bfull + s));
         ++t;
       }
-      // no copy may still be landing when the CTA exits
+      // no copy may still be landing when the CTA exits (Q included)
+      volatile int no_abort = 0;
+      if (is_k && !mbar_test(BAR(C::B_Q), 0)) mbar_wait(BAR(C::B_Q), 0, &no_abort, status, 2, kDrainLimit);
       for (int s = 0; s < NSLOT && s < t; ++s) {
         const int last = s + ((t - 1 - s) / NSLOT) * NSLOT;
-        if (!mbar_test(BAR(bfull + s), (last / NSLOT) & 1)) {
-          volatile int no_abort = 0;
-          mbar_wait(BAR(bfull + s), (last / NSLOT) & 1, &no_abort, status, 2, 1ll << 28);
-        }
+        if (!mbar_test(BAR(bfull + s), (last / NSLOT) & 1))
+          mbar_wait(BAR(bfull + s), (last / NSLOT) & 1, &no_abort, status, 2, kDrainLimit);
       }
     }
   } else if (warp == kSWarp) {
@@ -290,16 +293,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       StepIter it;
       it.init(tile_idx, tile_cnt, bh, nb, BLK, qt, status, false, token);
       constexpr uint32_t idq = idesc_bf16(BM, BN, 0);
-      bool ok = mbar_wait(BAR(C::B_Q), 0, abort_flag, status, 4);
+      bool ok = mbar_wait(BAR(C::B_Q), 0, abort_flag, status, 4, wait_limit);
       int j = 0, kt;
       uint32_t bits;
       while (ok && it.next(kt, bits)) {
         if (j >= 2) {   // buffer j%2 is free once its softmax group has read S_{j-2}
-          ok = mbar_wait(BAR(C::B_SFREE + (j & 1)), ((j - 2) >> 1) & 1, abort_flag, status, 5);
+          ok = mbar_wait(BAR(C::B_SFREE + (j & 1)), ((j - 2) >> 1) & 1, abort_flag, status, 5, wait_limit);
           if (!ok) break;
         }
         const int s = j % NSLOT;
-        ok = mbar_wait(BAR(C::B_KFULL + s), (j / NSLOT) & 1, abort_flag, status, 3);
+        ok = mbar_wait(BAR(C::B_KFULL + s), (j / NSLOT) & 1, abort_flag, status, 3, wait_limit);
         if (!ok) break;
         tc_fence_after();
         const uint32_t d = tmem + uint32_t(j & 1) * 128u;
@@ -314,6 +317,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(BAR(C::B_KEMPTY + s));
         ++j;
       }
+      // Every QK^T this lane issued has completed before the TMEM is released
+      // (after an abort some S_j may never have been read).
+      umma_commit(BAR(C::B_SDRAIN));
+      volatile int no_abort = 0;
+      mbar_wait(BAR(C::B_SDRAIN), 0, &no_abort, status, 11, kDrainLimit);
     }
   } else if (warp == kPVWarp) {
     // ------------------------------------------------------------ UMMA issuer: O += P V
@@ -326,8 +334,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t bits;
       while (ok && it.next(kt, bits)) {
         const int s = j % NSLOT;
-        ok = mbar_wait(BAR(C::B_VFULL + s), (j / NSLOT) & 1, abort_flag, status, 3) &&
-             mbar_wait(BAR(C::B_P + (j & 1)), (j >> 1) & 1, abort_flag, status, 6);
+        ok = mbar_wait(BAR(C::B_VFULL + s), (j / NSLOT) & 1, abort_flag, status, 3, wait_limit) &&
+             mbar_wait(BAR(C::B_P + (j & 1)), (j >> 1) & 1, abort_flag, status, 6, wait_limit);
         if (!ok) break;
         tc_fence_after();
         const uint32_t d = tmem + 256u + uint32_t(j & 1) * D;
@@ -345,6 +353,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         ++j;
       }
       umma_commit(BAR(C::B_O));
+      // every PV this lane issued has completed before the TMEM is released
+      volatile int no_abort = 0;
+      mbar_wait(BAR(C::B_O), 0, &no_abort, status, 12, kDrainLimit);
     }
   } else {
     // ------------------------------------------------------------ softmax groups
@@ -373,7 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       kt = kt_next;
       bits = bits_next;
       more = it.next(kt_next, bits_next) && it.next(kt_next, bits_next);
-      ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_S + grp), u & 1, abort_flag, status, 7));
+      ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_S + grp), u & 1, abort_flag, status, 7, wait_limit));
       if (!ok) break;
       tc_fence_after();
       uint32_t sr[4][32];
@@ -447,7 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float mref = m_use == -INFINITY ? 0.f : m_use;
       // this group's P tile and O accumulator are free once its PV of step j-2 completed
       if (u >= 1) {
-        ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_PV + grp), (u - 1) & 1, abort_flag, status, 8));
+        ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_PV + grp), (u - 1) & 1, abort_flag, status, 8, wait_limit));
         if (!ok) break;
       }
       // exp2 arguments and row sums two at a time (f32x2), P packed to bf16x2
@@ -497,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++u;
     }
     // ---- merge the two groups' partial results (every softmax thread gets here once)
-    const bool done = ok && __all_sync(0xffffffffu, mbar_wait(BAR(C::B_O), 0, abort_flag, status, 10));
+    const bool done = ok && __all_sync(0xffffffffu, mbar_wait(BAR(C::B_O), 0, abort_flag, status, 10, wait_limit));
     // all UMMAs have completed: the P tiles are free and hold the exchange
     float* xch = reinterpret_cast<float*>(gbase + C::OFF_P);
     xch[grp * 256 + r] = done ? m_use : -INFINITY;
@@ -562,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D, int BLK, bool TOKEN>
 cudaError_t launch_tc(const crisp_params& p, const void* q, const void* k, const void* v,
                       const int32_t* tile_idx, const int32_t* tile_cnt, void* o, float* lse, void* ws,
-                      cudaStream_t st) {
+                      cudaStream_t st, long long wait_limit) {
   CUtensorMap mq, mk, mv;
   const uint64_t N = uint64_t(p.seqlen);
   if (!make_tmap(&mq, q, uint64_t(p.batch) * p.h_q * N, D) || !make_tmap(&mk, k, uint64_t(p.batch) * p.h_kv * N, D) ||
@@ -573,7 +584,7 @@ cudaError_t launch_tc(const crisp_params& p, const void* q, const void* k, const
   if (e != cudaSuccess) return e;
   const unsigned grid = unsigned(p.batch) * p.h_q * ((p.seqlen + BM - 1) / BM);
   kern<<<grid, kThreads, Cfg<D>::SMEM, st>>>(mq, mk, mv, tile_idx, tile_cnt, static_cast<__nv_bfloat16*>(o),
-                                             lse, p, ws);
+                                             lse, p, ws, wait_limit);
   return cudaGetLastError();
 }
 
@@ -581,17 +592,18 @@ cudaError_t launch_tc(const crisp_params& p, const void* q, const void* k, const
 
 cudaError_t run_attention(const crisp_params& p, const void* q, const void* k, const void* v,
                           const int32_t* tile_idx, const int32_t* tile_cnt, void* o, float* lse,
-                          void* ws, cudaStream_t st) {
+                          void* ws, cudaStream_t st, long long wait_limit) {
   // token-granular lists carry per-tile flags (block 128 only, checked by the ABI)
   const bool token = tile_idx && p.vs_granularity == CRISP_GRAN_TOKEN && p.block == 128;
+  const long long wl = wait_limit;
   if (p.head_dim == 64) {
-    if (token) return launch_tc<64, 128, true>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st);
-    return p.block == 64 ? launch_tc<64, 64, false>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st)
-                         : launch_tc<64, 128, false>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st);
+    if (token) return launch_tc<64, 128, true>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st, wl);
+    return p.block == 64 ? launch_tc<64, 64, false>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st, wl)
+                         : launch_tc<64, 128, false>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st, wl);
   }
-  if (token) return launch_tc<128, 128, true>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st);
-  return p.block == 64 ? launch_tc<128, 64, false>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st)
-                       : launch_tc<128, 128, false>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st);
+  if (token) return launch_tc<128, 128, true>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st, wl);
+  return p.block == 64 ? launch_tc<128, 64, false>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st, wl)
+                       : launch_tc<128, 128, false>(p, q, k, v, tile_idx, tile_cnt, o, lse, ws, st, wl);
 }
 
 }  // namespace crisp

@@ -19,9 +19,13 @@
 //    wrong results — order them on one stream;
 //  * problems whose routing scratch exceeds the array are rejected with
 //    CRISP_ERR_WORKSPACE before anything is launched;
-//  * the first call on a device looks up the array's device address (one
-//    cudaGetSymbolAddress per device, with that device current), so make
-//    that first call before any stream capture.
+//  * each call outside stream capture looks up the array's device address
+//    (cudaGetSymbolAddress, with the device current); during capture the
+//    address of the last lookup on that device is used, so make the first
+//    call on a device before any stream capture;
+//  * kernel-side errors (a bounded wait that ran out, an out-of-range
+//    sequence length) land in a status word at the start of the array:
+//    crisp_get_device_status(NULL, ...) reads and clears it.
 #include <mutex>
 
 #include "common.cuh"
@@ -40,21 +44,29 @@ constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
-// Device address of g_route_scratch on the current device, looked up once.
-int scratch_address(void** out) {
+}  // namespace
+
+// Device address of g_route_scratch on the current device. Outside stream
+// capture it is looked up on every call (a context that was reset and created
+// again may have loaded the module at another address); during capture, when
+// no lookup may run, the address cached by the last lookup on this device is
+// used, so the first call on a device must come before any capture.
+int crisp::noalloc_scratch(void** out, cudaStream_t st) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return CRISP_ERR_CUDA;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return CRISP_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
+  if (cap == cudaStreamCaptureStatusNone) {
     void* addr = nullptr;
     if (cudaGetSymbolAddress(&addr, g_route_scratch) != cudaSuccess || !addr) return CRISP_ERR_CUDA;
     g_scratch_addr[dev] = addr;
   }
+  if (!g_scratch_addr[dev]) return CRISP_ERR_CUDA;
   *out = g_scratch_addr[dev];
   return CRISP_OK;
 }
 
-}  // namespace
 
 extern "C" int crisp_route_noalloc(const crisp_params* p, const void* q, const void* k,
                                    int32_t* pattern, float* score, float* p_v, float* p_s,
@@ -69,10 +81,10 @@ extern "C" int crisp_route_noalloc(const crisp_params* p, const void* q, const v
   // before the pooled-query region.
   const size_t need = make_workspace(*p).qbar;
   if (need > size_t(CRISP_NOALLOC_SCRATCH_BYTES)) return CRISP_ERR_WORKSPACE;
-  void* scratch = nullptr;
-  const int a = scratch_address(&scratch);
-  if (a != CRISP_OK) return a;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* scratch = nullptr;
+  const int a = noalloc_scratch(&scratch, st);
+  if (a != CRISP_OK) return a;
   // The status word and the per-head completion counters must start at zero;
   // every other scratch byte the routing kernels read is written earlier in
   // the same call.

@@ -1,5 +1,5 @@
-// Proxy attention statistics (CRISP paper, Algorithm 2 and Algorithm 3 lines
-// 3-5) on the 5th-generation tensor cores of sm_100a.
+// Proxy attention statistics (CRISP paper, Algorithm 2, and the block scores
+// that Algorithm 3 thresholds) on the 5th-generation tensor cores of sm_100a.
 //
 // The proxy rows are the last R = block query rows of a head. For every proxy
 // row r and key tile kb this kernel writes the tile-local row max m (log2
@@ -24,7 +24,8 @@
 //                      diagonal.
 // Two CTAs fit on an SM (256 TMEM columns and < 100 KB shared memory each).
 // Every mbarrier wait is bounded (status CRISP_ERR_TIMEOUT and a CTA abort
-// flag on expiry); the producer drains its copies before the CTA exits.
+// flag on expiry); the producer drains its copies and the issuer waits for a
+// final commit of its UMMAs before the TMEM is released and the CTA exits.
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -50,7 +51,7 @@ struct PxCfg {
   static constexpr int OFF_XCH = OFF_RING + NSLOT * T_BYTES;    // float[2 groups][2][PM]
   static constexpr int OFF_BAR = OFF_XCH + 2 * 2 * PM * 4;
   static constexpr int B_Q = 0, B_KFULL = 1, B_KEMPTY = 1 + NSLOT, B_S = 1 + 2 * NSLOT, B_SFREE = B_S + 2,
-                       N_BARS = B_SFREE + 2;
+                       B_DRAIN = B_SFREE + 2, N_BARS = B_DRAIN + 1;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * N_BARS;
   static constexpr int OFF_ABORT = OFF_TMEM + 8;
   static constexpr int SMEM = OFF_ABORT + 8 + 1024;   // + alignment slack
@@ -84,7 +85,7 @@ __device__ __noinline__ void merge_chunks(const crisp_params& p, void* ws, int b
 template <int D, int R>
 __global__ void __launch_bounds__(kPxThreads, 2)
     proxy_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
-                    crisp_params p, void* ws) {
+                    crisp_params p, void* ws, long long wait_limit) {
   using C = PxCfg<D>;
   constexpr int NSLOT = C::NSLOT;
   constexpr int KPS = PN / R;          // key tiles per step
@@ -130,6 +131,7 @@ __global__ void __launch_bounds__(kPxThreads, 2)
       mbar_init(BAR(C::B_S + i), 1);
       mbar_init(BAR(C::B_SFREE + i), R / 32);   // one arrival per warp holding proxy rows
     }
+    mbar_init(BAR(C::B_DRAIN), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -154,7 +156,7 @@ __global__ void __launch_bounds__(kPxThreads, 2)
       int j = 0;
       for (; j < nsteps; ++j) {
         const int s = j % NSLOT, u = j / NSLOT;
-        if (u >= 1 && !mbar_wait(BAR(C::B_KEMPTY + s), (u - 1) & 1, abort_flag, status, 21)) break;
+        if (u >= 1 && !mbar_wait(BAR(C::B_KEMPTY + s), (u - 1) & 1, abort_flag, status, 21, wait_limit)) break;
         mbar_arrive_expect_tx(BAR(C::B_KFULL + s), C::T_BYTES);
         for (int box = 0; box < D / 64; ++box)
           tma_load_2d(sRing + s * C::T_BYTES + box * PN * 128, &tmk, box * 64, k_row0 + j * PN,
@@ -162,25 +164,25 @@ __global__ void __launch_bounds__(kPxThreads, 2)
       }
       // no copy may still be landing when the CTA exits
       volatile int no_abort = 0;
-      if (!mbar_test(BAR(C::B_Q), 0)) mbar_wait(BAR(C::B_Q), 0, &no_abort, status, 22, 1ll << 28);
+      if (!mbar_test(BAR(C::B_Q), 0)) mbar_wait(BAR(C::B_Q), 0, &no_abort, status, 22, kDrainLimit);
       for (int s = 0; s < NSLOT && s < j; ++s) {
         const int last = s + ((j - 1 - s) / NSLOT) * NSLOT;
         if (!mbar_test(BAR(C::B_KFULL + s), (last / NSLOT) & 1))
-          mbar_wait(BAR(C::B_KFULL + s), (last / NSLOT) & 1, &no_abort, status, 22, 1ll << 28);
+          mbar_wait(BAR(C::B_KFULL + s), (last / NSLOT) & 1, &no_abort, status, 22, kDrainLimit);
       }
     }
   } else if (warp == kPxMma) {
     // ------------------------------------------------------------ UMMA issuer
     if (lane == 0) {
       constexpr uint32_t idq = idesc_bf16(PM, PN, 0);
-      bool ok = mbar_wait(BAR(C::B_Q), 0, abort_flag, status, 23);
+      bool ok = mbar_wait(BAR(C::B_Q), 0, abort_flag, status, 23, wait_limit);
       for (int j = 0; ok && j < nsteps; ++j) {
         if (j >= 2) {   // buffer j%2 is free once its group has read S_{j-2}
-          ok = mbar_wait(BAR(C::B_SFREE + (j & 1)), ((j - 2) >> 1) & 1, abort_flag, status, 24);
+          ok = mbar_wait(BAR(C::B_SFREE + (j & 1)), ((j - 2) >> 1) & 1, abort_flag, status, 24, wait_limit);
           if (!ok) break;
         }
         const int s = j % NSLOT;
-        ok = mbar_wait(BAR(C::B_KFULL + s), (j / NSLOT) & 1, abort_flag, status, 25);
+        ok = mbar_wait(BAR(C::B_KFULL + s), (j / NSLOT) & 1, abort_flag, status, 25, wait_limit);
         if (!ok) break;
         tc_fence_after();
         const uint32_t d = tmem + uint32_t(j & 1) * 128u;
@@ -194,6 +196,11 @@ __global__ void __launch_bounds__(kPxThreads, 2)
         umma_commit(BAR(C::B_S + (j & 1)));
         umma_commit(BAR(C::B_KEMPTY + s));
       }
+      // Every UMMA issued here has completed before the TMEM is released
+      // (after an abort some S_j may never have been read).
+      umma_commit(BAR(C::B_DRAIN));
+      volatile int no_abort = 0;
+      mbar_wait(BAR(C::B_DRAIN), 0, &no_abort, status, 27, kDrainLimit);
     }
   } else if ((warp & 3) * 32 >= ROW0) {
     // ------------------------------------------------------------ row statistics
@@ -275,7 +282,7 @@ __global__ void __launch_bounds__(kPxThreads, 2)
 
     int u = 0;
     for (int j = grp; j < nsteps; j += 2, ++u) {
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_S + grp), u & 1, abort_flag, status, 26));
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(BAR(C::B_S + grp), u & 1, abort_flag, status, 26, wait_limit));
       if (!ok) break;
       tc_fence_after();
       const int kbs = kb0 + j * KPS;
@@ -404,7 +411,8 @@ __global__ void __launch_bounds__(kPxThreads, 2)
 }
 
 template <int D, int R>
-cudaError_t launch_proxy(const crisp_params& p, const void* q, const void* k, void* ws, cudaStream_t st) {
+cudaError_t launch_proxy(const crisp_params& p, const void* q, const void* k, void* ws, cudaStream_t st,
+                         long long wait_limit) {
   CUtensorMap mq, mk;
   const uint64_t N = uint64_t(p.seqlen);
   if (!make_tmap(&mq, q, uint64_t(p.batch) * p.h_q * N, D) || !make_tmap(&mk, k, uint64_t(p.batch) * p.h_kv * N, D))
@@ -415,16 +423,18 @@ cudaError_t launch_proxy(const crisp_params& p, const void* q, const void* k, vo
   const int nb = n_blocks(p);
   const int nc = (nb + proxy_chunk(p) - 1) / proxy_chunk(p);
   const unsigned grid = unsigned(p.batch) * p.h_q * nc;
-  kern<<<grid, kPxThreads, PxCfg<D>::SMEM, st>>>(mq, mk, p, ws);
+  kern<<<grid, kPxThreads, PxCfg<D>::SMEM, st>>>(mq, mk, p, ws, wait_limit);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t run_proxy_stats(const crisp_params& p, const void* q, const void* k, void* ws, cudaStream_t st) {
+cudaError_t run_proxy_stats(const crisp_params& p, const void* q, const void* k, void* ws, cudaStream_t st,
+                            long long wait_limit) {
+  const long long wl = wait_limit;
   if (p.head_dim == 64)
-    return p.block == 64 ? launch_proxy<64, 64>(p, q, k, ws, st) : launch_proxy<64, 128>(p, q, k, ws, st);
-  return p.block == 64 ? launch_proxy<128, 64>(p, q, k, ws, st) : launch_proxy<128, 128>(p, q, k, ws, st);
+    return p.block == 64 ? launch_proxy<64, 64>(p, q, k, ws, st, wl) : launch_proxy<64, 128>(p, q, k, ws, st, wl);
+  return p.block == 64 ? launch_proxy<128, 64>(p, q, k, ws, st, wl) : launch_proxy<128, 128>(p, q, k, ws, st, wl);
 }
 
 }  // namespace crisp

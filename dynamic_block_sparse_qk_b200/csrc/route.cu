@@ -1,6 +1,6 @@
 // PatSearch (CRISP paper, Algorithm 2) on sm_100a: proxy attention of the
 // last query block against all keys, its vertical / slash block scores
-// (Algorithm 3 lines 3-5), C_struct (Eq. 2) and the JSD router of the
+// (the scores Algorithm 3 thresholds), C_struct (Eq. 2) and the JSD router of the
 // paper's Appendix A (Algorithm 5).
 //
 // The b x n proxy map is never stored. One tensor-core pass (proxy_sm100.cu)
@@ -75,7 +75,7 @@ __global__ void proxy_scores_kernel(crisp_params p, void* ws, float* __restrict_
 }
 
 // ---------------------------------------------------------------------------
-// Block-mean pooling (Algorithm 4 line 3; Algorithm 5 line 3): a block of
+// Block-mean pooling (Algorithms 4 and 5): a block of
 // one head per CTA step (16-byte loads, rows split across thread groups,
 // smem reduce), grid-stride over blocks. One launch covers K and Q: heads
 // y < nk are K heads (skipped unless a query head of the group is PE, or
@@ -235,13 +235,14 @@ cudaError_t launch_pool(const crisp_params& p, const void* k, const void* q, int
 }
 
 cudaError_t run_route(const crisp_params& p, const void* q, const void* k, void* ws,
-                      int32_t* pattern, float* score, float* p_v, float* p_s, cudaStream_t st) {
+                      int32_t* pattern, float* score, float* p_v, float* p_s, cudaStream_t st,
+                      long long wait_limit) {
   const Workspace W = make_workspace(p);
   const int nb = n_blocks(p);
   const int BH = p.batch * p.h_q;
   // proxy statistics (+ row merge in the last CTA of each head), block
   // scores (+ C_struct route by the warp that computes p_v[0])
-  cudaError_t e = run_proxy_stats(p, q, k, ws, st);
+  cudaError_t e = run_proxy_stats(p, q, k, ws, st, wait_limit);
   if (e != cudaSuccess) return e;
   proxy_scores_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, ws, p_v, p_s, pattern, score);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

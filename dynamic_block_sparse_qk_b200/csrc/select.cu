@@ -145,11 +145,12 @@ __global__ void __launch_bounds__(1024) vs_select_kernel(crisp_params p, const i
 }
 
 // ---------------------------------------------------------------------------
-// PE estimate (Algorithm 4 line 4): logits of Q_bar K_bar^T for kb <= qb,
+// PE estimate (Algorithm 4): logits of Q_bar K_bar^T for kb <= qb,
 // 64x64 tiles (grid-stride over PE heads and tiles), fp32 FMA; written in
 // log2 units into abar together
 // with per-(row, tile) max / sum partials. Then a row pass normalises and
-// divides by N_b (Algorithm 4 line 6: the total of N_b causal rows is N_b).
+// divides by N_b (Algorithm 4 normalises by the total, which for N_b causal
+// softmax rows is N_b).
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) pe_logits_kernel(crisp_params p, const int32_t* pattern,

@@ -41,17 +41,26 @@ __device__ inline bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Cycle limit of the pipelined kernels' waits (about a second at the B200's
+// clocks), and the limit of the waits that drain copies and tensor-core
+// operations already in flight before a CTA exits.
+constexpr long long kWaitLimit = 1ll << 31;
+constexpr long long kDrainLimit = 1ll << 28;
+
 // Bounded wait for the phase with the given parity. Gives up when the CTA's
 // abort flag is raised or after `limit` clock cycles; on a timeout it records
 // CRISP_ERR_TIMEOUT (with `where`) in the status word and raises the abort
-// flag so the other roles leave their loops too.
+// flag so the other roles leave their loops too. The clock and the flag are
+// read every 256 probes, or on every probe when the limit is short (below
+// 2^20 cycles: the diagnostic entry points that make waits run out).
 __device__ inline bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                 int32_t* status, int where, long long limit = (1ll << 31)) {
+                                 int32_t* status, int where, long long limit = kWaitLimit) {
   if (mbar_test(bar, parity)) return true;
   const long long t0 = clock64();
+  const uint32_t every = limit < (1ll << 20) ? 0u : 255u;
   for (uint32_t it = 1;; ++it) {
     if (mbar_test(bar, parity)) return true;
-    if ((it & 255u) == 0) {
+    if ((it & every) == 0) {
       if (*abort) return false;
       if (clock64() - t0 > limit) {
         report_error(status, CRISP_ERR_TIMEOUT, where);

@@ -90,7 +90,7 @@ typedef struct {
   float gamma;         /* cumulative coverage of Algorithms 4 and 6, in (0, 1] */
   float tau_proxy;     /* C_struct routing threshold of Algorithm 2 */
   float tau_jsd;       /* JSD routing threshold of Algorithm 5 (not given by the paper) */
-  int32_t k_min_blocks;/* minimum blocks per VS direction (Algorithm 3 line 11), >= 1 */
+  int32_t k_min_blocks;/* minimum blocks per VS direction (k_min of Algorithm 3), >= 1 */
   int32_t router;      /* crisp_router */
   int32_t vs_rule;     /* crisp_vs_rule */
   float sm_scale;      /* softmax scale; 0 selects 1/sqrt(head_dim) */
@@ -182,8 +182,13 @@ int crisp_dense_prefill(const crisp_params* p, const void* q, const void* k, con
  *  - All calls on a device share the array, which keeps the last call's
  *    contents; calls whose kernels overlap on the GPU race. Issue them in
  *    order on one stream.
- *  - The first call on each device looks up the array's address (with that
- *    device current); make that first call before any stream capture. */
+ *  - Each call outside stream capture looks up the array's address (with
+ *    the device current); during capture the address of the last lookup on
+ *    that device is used, so make the first call on a device before any
+ *    stream capture.
+ *  - Kernel-side errors (a bounded wait that ran out, an out-of-range entry
+ *    of seq_lens) are recorded in a status word at the start of the array;
+ *    read and clear it with crisp_get_device_status(NULL, ...). */
 #define CRISP_NOALLOC_SCRATCH_BYTES (16u << 20)
 int crisp_route_noalloc(const crisp_params* p, const void* q, const void* k, int32_t* pattern,
                         float* score, float* p_v, float* p_s, void* stream);
@@ -197,9 +202,26 @@ int crisp_route_noalloc(const crisp_params* p, const void* q, const void* k, int
  * CRISP_ERR_ARG for a bad workspace or limit. The paper has no counterpart. */
 int crisp_selftest_wait_timeout(void* ws, long long limit_cycles, void* stream);
 
+/* Diagnostic: runs the two pipelined tensor-core kernels of a prefill — the
+ * proxy statistics kernel of crisp_route and the attention kernel of
+ * crisp_dense_prefill — on the given problem with every pipeline wait cut to
+ * `limit_cycles` (1 .. 2^20 - 1) SM clock cycles, short enough that waits run
+ * out. A CTA whose wait runs out records CRISP_ERR_TIMEOUT in the status word
+ * of `ws`, leaves its loops, waits (bounded) for the copies and tensor-core
+ * operations it has in flight, releases its tensor memory and returns; the
+ * context stays usable and the next call of any entry point runs normally.
+ * `o` and the routing scratch of `ws` hold unspecified values afterwards.
+ * Arguments as for crisp_dense_prefill (validated the same way; a limit out
+ * of range returns CRISP_ERR_ARG). The paper has no counterpart. */
+int crisp_selftest_pipeline_timeout(const crisp_params* p, const void* q, const void* k, const void* v,
+                                    void* o, void* ws, size_t ws_bytes, long long limit_cycles,
+                                    void* stream);
+
 /* Synchronises `stream`, copies the device status word out of `ws` into
  * *status (CRISP_OK or CRISP_ERR_TIMEOUT / CRISP_ERR_DEVICE) and clears it.
- * Returns CRISP_OK unless the copy itself failed. */
+ * ws == NULL reads the status word of crisp_route_noalloc's scratch array on
+ * the current device. Returns CRISP_OK unless the copy itself failed
+ * (CRISP_ERR_CUDA) or status is NULL / ws misaligned (CRISP_ERR_ARG). */
 int crisp_get_device_status(void* ws, int32_t* status, void* stream);
 
 #ifdef __cplusplus

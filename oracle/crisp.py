@@ -69,12 +69,12 @@ def bf16_to_f64(t) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
-# (a) Proxy attention — CRISP paper, Algorithm 2 (PatSearch), lines 3-5.
+# (a) Proxy attention — CRISP paper, Algorithm 2 (PatSearch): the proxy map.
 # ---------------------------------------------------------------------------
 def proxy_attention(q_hat: np.ndarray, k: np.ndarray, scale: float) -> np.ndarray:
     """A_hat = Softmax(Q_hat K^T * scale) with causal masking.
 
-    q_hat: [b, d] — the last b query rows (Algorithm 2, line 3).
+    q_hat: [b, d] — the last b query rows (the representative block of Algorithm 2).
     k:     [n, d] — all keys.  Row r of q_hat is at position n - b + r and
     sees keys j <= n - b + r (reading: causal prefill).
     Returns [b, n] float64; masked entries are exactly 0.
@@ -104,7 +104,7 @@ def _block_sums(x: np.ndarray, block: int) -> np.ndarray:
 
 
 def vertical_slash_scores(a_hat: np.ndarray, block: int):
-    """Block scores p_v, p_s of Algorithm 3, lines 3-5.
+    """Block scores p_v (vertical) and p_s (slash) that Algorithm 3 thresholds.
 
     a_v = colmean(A_hat): mean over the b proxy rows of each key column.
     a_s = diagmean(A_hat): mean over rows of the entries on each diagonal,
@@ -137,7 +137,7 @@ def c_struct_from_map(a_hat: np.ndarray, block: int) -> float:
 
 
 def route_cstruct(c: float, tau: float) -> int:
-    """Algorithm 2, lines 9-13: VS iff C_struct >= tau_proxy (float32 compare)."""
+    """The routing rule of Algorithm 2 with Eq. 2: VS iff C_struct >= tau_proxy (float32 compare)."""
     return VS if np.float32(c) >= np.float32(tau) else PE
 
 
@@ -145,7 +145,7 @@ def route_cstruct(c: float, tau: float) -> int:
 # JSD router (comparison path) — CRISP paper, Appendix A, Algorithm 5.
 # ---------------------------------------------------------------------------
 def pooled_estimate_last_block(q_hat: np.ndarray, k: np.ndarray, block: int, scale: float):
-    """a_bar = Softmax(pool(Q_hat) pool(K)^T * scale) over all key blocks (line 3).
+    """a_bar = Softmax(pool(Q_hat) pool(K)^T * scale) over all key blocks (Algorithm 5).
 
     pool = block mean. The last query block sees every key block, so no
     block-level causal mask applies.
@@ -164,7 +164,8 @@ def _kl(p: np.ndarray, m: np.ndarray) -> float:
 
 
 def js_distance(a_hat: np.ndarray, a_bar: np.ndarray) -> float:
-    """Algorithm 5, line 5: D_JS = sqrt(KL(a_hat||m)/2 + KL(a_bar||m)/2), m = mean.
+    """The Jensen-Shannon distance of Algorithm 5: D_JS = sqrt(KL(a_hat||m)/2 + KL(a_bar||m)/2),
+    m the mean of the two distributions.
 
     Natural logarithm; 0*log(0) = 0.
     """
@@ -173,7 +174,7 @@ def js_distance(a_hat: np.ndarray, a_bar: np.ndarray) -> float:
 
 
 def route_jsd(djs: float, tau: float) -> int:
-    """Algorithm 5, lines 6-10: VS iff D_JS >= tau (float32 compare)."""
+    """The routing rule of Algorithm 5: VS iff D_JS >= tau (float32 compare)."""
     return VS if np.float32(djs) >= np.float32(tau) else PE
 
 
@@ -181,7 +182,7 @@ def route_jsd(djs: float, tau: float) -> int:
 # (b) Sink-aware vertical-slash selection — Algorithm 3, Eq. 3 and Eq. 4.
 # ---------------------------------------------------------------------------
 def noise_floor(p: np.ndarray) -> np.float32:
-    """Eq. 3 / Algorithm 3 lines 7-8: mu = max(1 - p[0] - p[N_b-1], 0) / (N_b - 2)."""
+    """Eq. 3: the mean mass of the non-retained blocks, mu = max(1 - p[0] - p[N_b-1], 0) / (N_b - 2)."""
     p32 = p.astype(np.float32)
     nb = p32.shape[0]
     r = np.float32(1.0) - p32[0] - p32[nb - 1]
@@ -213,7 +214,7 @@ def _topk_desc(values32: np.ndarray, k: int) -> np.ndarray:
 
 
 def vs_index_alpha(p: np.ndarray, alpha: float, k_min: int, floor: str = "mean") -> np.ndarray:
-    """Algorithm 3, lines 7-12 for one direction.
+    """The sink-aware index of Algorithm 3 (Eq. 3-4) for one direction.
 
     k_d = #{j : p[j] > alpha * mu} over all blocks (Eq. 4, strict),
     clipped to [k_min, N_b]; S_d = top-k_d(p). Returns sorted block ids.
@@ -239,7 +240,7 @@ def _gamma_count(sorted_desc32: np.ndarray, gamma: float) -> int:
 def vs_index_gamma(p: np.ndarray, gamma: float, k_min: int) -> np.ndarray:
     """Appendix A, Algorithm 6, one direction: sort descending, accumulate to gamma.
 
-    p is already normalised (Algorithm 6 lines 2-3 divide by the total mass,
+    p is already normalised (Algorithm 6 divides by the total mass,
     which p_v / p_s carry as 1). Reading: the same k_min floor as
     Algorithm 3, so the two rules differ only in the budget.
     """
@@ -255,7 +256,7 @@ def vs_index_gamma(p: np.ndarray, gamma: float, k_min: int) -> np.ndarray:
 # (c) Pooled estimation for diffuse heads — Algorithm 4 (PE Index).
 # ---------------------------------------------------------------------------
 def pe_pool(x: np.ndarray, block: int) -> np.ndarray:
-    """Algorithm 4, line 3: block-mean pooling over all rows ([n, d] -> [N_b, d]);
+    """The block-mean pooling of Algorithm 4 ([n, d] -> [N_b, d]);
     a partial last block is the mean of the rows it holds."""
     n = x.shape[0]
     counts = np.minimum(block, n - block * np.arange(n_blocks(n, block)))
@@ -263,7 +264,7 @@ def pe_pool(x: np.ndarray, block: int) -> np.ndarray:
 
 
 def pe_estimate(q_bar: np.ndarray, k_bar: np.ndarray, scale: float) -> np.ndarray:
-    """Algorithm 4, line 4: A_bar = Softmax(Q_bar K_bar^T * scale).
+    """The pooled estimate of Algorithm 4: A_bar = Softmax(Q_bar K_bar^T * scale).
 
     Reading: causal at block level (query block i sees key blocks j <= i).
     Returns [N_b, N_b]; entries above the diagonal are 0.
@@ -277,7 +278,8 @@ def pe_estimate(q_bar: np.ndarray, k_bar: np.ndarray, scale: float) -> np.ndarra
 
 
 def pe_index(a_bar: np.ndarray, gamma: float) -> np.ndarray:
-    """Algorithm 4, lines 6-10: normalise, flatten, sort descending, gamma-cumsum.
+    """The gamma cut of Algorithm 4: the smallest set of largest normalised entries
+    whose mass reaches gamma.
 
     Flattening covers the causal (lower-triangle) entries in row-major order;
     flat id = i * N_b + j. Equal values -> lower flat id first.

@@ -92,7 +92,14 @@ def test_entry_points_validate_before_launch(lib):
     bad = _p(block=96)
     assert lib.crisp_dense_prefill(ctypes.byref(bad), fake, fake, fake, fake, None, fake, need, None) == -2
     st = ctypes.c_int32(0)
-    assert lib.crisp_get_device_status(None, ctypes.byref(st), None) == -1
+    assert lib.crisp_get_device_status(fake, None, None) == -1
+    assert lib.crisp_get_device_status(ctypes.c_void_p((1 << 20) + 8), ctypes.byref(st), None) == -1
+    assert lib.crisp_selftest_pipeline_timeout(ctypes.byref(p), fake, fake, fake, fake, fake, need, 0, None) == -1
+    assert lib.crisp_selftest_pipeline_timeout(ctypes.byref(p), fake, fake, fake, fake, fake, need, 1 << 20,
+                                               None) == -1
+    assert lib.crisp_selftest_pipeline_timeout(ctypes.byref(p), fake, fake, fake, None, fake, need, 64, None) == -1
+    assert lib.crisp_selftest_pipeline_timeout(ctypes.byref(p), fake, fake, fake, fake, fake, need - 1, 64,
+                                               None) == -3
 
 
 def test_selftest_validates_before_launch(lib):

@@ -403,7 +403,7 @@ def test_ragged_block_scores_bruteforce():
 
 
 def test_ragged_pooled_estimate_bruteforce():
-    # Algorithm 5 line 3 on a partial last block: the block means of K run over
+    # The block means of Algorithm 5 on a partial last block: the block means of K run over
     # the keys each block holds; the estimate is a softmax over all N_b blocks
     rng = _rng(27)
     B, n, d = 8, 8 * 5 + 3, 4

@@ -7,7 +7,9 @@ fixed scratch array compiled into the library. These tests call the new entry
 point through the C ABI and check it against crisp_route, which uses a
 caller workspace: equal patterns, scores and block scores (within the
 tolerance of the other parity tests) on consecutive calls that share the
-array, and a clean rejection of problems too large for it.
+array, a clean rejection of problems too large for it, and that a device-side
+error of a call lands in the array's status word, which
+crisp_get_device_status(NULL) reads and clears.
 """
 import ctypes
 
@@ -87,3 +89,21 @@ def test_largest_supported_problem_and_rejection(lib):
     big = lib.make_params(1, 32, 8, 65536, 128, block=128)
     z = ctypes.c_void_p(1 << 20)
     assert lib.load_library().crisp_route_noalloc(ctypes.byref(big), z, z, z, z, z, z, None) == -3
+
+
+def test_device_errors_reach_the_status_reader(lib):
+    # a sequence length below 2 * block + 1 is clamped by the kernels and
+    # reported as CRISP_ERR_DEVICE in the array's status word; the reader with
+    # a NULL workspace returns it once and clears it
+    w = WORKLOADS["tiny"]
+    q, k, _, _ = make_qkv(w)
+    q, k = q.cuda(), k.cuda()
+    assert lib.crisp_get_device_status(None) == 0                 # whatever an earlier call left
+    lens = torch.tensor([2 * w.block], dtype=torch.int32, device="cuda")
+    p = lib.params_for(q, k, block=w.block, seq_lens=lens)
+    _via_noalloc_cabi(lib, p, q, k)
+    assert lib.crisp_get_device_status(None) == -6                # CRISP_ERR_DEVICE
+    assert lib.crisp_get_device_status(None) == 0
+    ok = lib.params_for(q, k, block=w.block)
+    _same(_via_noalloc_cabi(lib, ok, q, k), _via_workspace(lib, ok, q, k))
+    assert lib.crisp_get_device_status(None) == 0
