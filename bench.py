@@ -132,24 +132,27 @@ def workload_config(w, args) -> dict:
             **({"lengths": list(w.lengths)} if w.lengths is not None else {})}
 
 
-def stage_algorithmic_bytes(w, pattern) -> dict:
+def stage_algorithmic_bytes(w, pattern, tiles: int) -> dict:
     """HBM bytes the routing and selection stages must move at least once
-    (algorithmic, not measured): routing reads K once per KV head (the proxy
+    (algorithmic, not measured). Routing reads K once per KV head (the proxy
     is bound by its exp2 work, so this only says how far from HBM-bound it
-    is); selection pools K of the KV heads with a PE query head and Q of the
-    PE heads, then passes over each PE head's N_b(N_b+1)/2 estimate entries
-    (fp32) seven times: written by the logits, read and written by the
-    normalisation, read by three radix levels, the tie count and the tile
-    builder."""
+    is). Selection reads Q of the PE heads and K of the KV heads with a PE
+    query head once (block-mean pooling), passes once over each PE head's
+    N_b(N_b+1)/2 fp32 estimate entries (the gamma cut), and writes the tile
+    lists: 4 bytes per executed tile and per query block (counts). The
+    kernels pass over the estimate more than once (logits, normalisation,
+    three radix levels, ties, tile builder); those repeats are the
+    implementation's, not the algorithm's, and are not counted."""
     g = w.h_q // w.h_kv
     d2 = w.head_dim * 2
     route = sum(w.length(b) * w.h_kv * d2 for b in range(w.batch))
-    select = 0
+    select = 4 * int(tiles)
     for b in range(w.batch):
         n = w.length(b)
         nb = -(-n // w.block)
         pe = [h for h in range(w.h_q) if pattern[b * w.h_q + h] == 1]
-        select += (len(pe) + len({h // g for h in pe})) * n * d2 + len(pe) * nb * (nb + 1) // 2 * 4 * 7
+        select += (len(pe) + len({h // g for h in pe})) * n * d2 + len(pe) * nb * (nb + 1) // 2 * 4
+        select += w.h_q * nb * 4
     return {"route": route, "select": select}
 
 
@@ -203,7 +206,7 @@ def run_ours(args, rank, world, local_rank):
     n_vs = int((pattern == 0).sum().item())
     nbv = [-(-w.length(b) // w.block) for b in range(w.batch)]        # each sequence's blocks
     causal_tiles = p.h_q * sum(x * (x + 1) // 2 for x in nbv)
-    stage_bytes = stage_algorithmic_bytes(w, pattern.cpu().tolist())
+    stage_bytes = stage_algorithmic_bytes(w, pattern.cpu().tolist(), cnt_sum)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     if world > 1:
@@ -321,6 +324,105 @@ def run_ours(args, rank, world, local_rank):
 
 
 # ----------------------------------------------------------------------------- sweep
+def time_point(C, p, q, k, v, ws, timed, dev) -> dict:
+    """Per-stage CUDA-event times of one prefill configuration (route,
+    select, attend; each the mean of timed()'s repetitions), its tile
+    density and the attention kernel's TFLOP/s on executed tiles."""
+    import torch
+    out = {}
+
+    def route():
+        out["r"] = C.crisp_route(p, q, k, ws)
+
+    def select():
+        r = out["r"]
+        out["s"] = C.crisp_select(p, q, k, r[0], r[2], r[3], ws, want_mask=False)
+
+    def attend():
+        s_ = out["s"]
+        out["a"] = C.crisp_sparse_prefill(p, q, k, v, s_[1], s_[2], ws, want_lse=False)
+
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        t_route = timed(route)
+        t_select = timed(select)
+        t_attend = timed(attend)
+    pattern, tcnt = out["r"][0], out["s"][2]
+    nb = p.n_blocks
+    causal = p.batch * p.h_q * nb * (nb + 1) // 2
+    tiles = int(tcnt.sum())
+    status = C.crisp_get_device_status(ws)
+    return {"route_ms": round(t_route, 4), "select_ms": round(t_select, 4), "attend_ms": round(t_attend, 4),
+            "total_ms": round(t_route + t_select + t_attend, 4), "density": round(tiles / causal, 5),
+            "executed_tiles": tiles, "vs_heads": int((pattern == 0).sum()), "heads": p.batch * p.h_q,
+            "attend_tflops": round(tiles * 4 * p.block ** 2 * p.head_dim / (t_attend * 1e-3) / 1e12, 1),
+            "device_status": status, "clocks": clk.summary(), "_pattern": pattern.clone()}
+
+
+def _event_timer(dev, reps):
+    import torch
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / reps
+    return timed
+
+
+# The pages' latency comparison (CRISP page, Section 5.3 and Table 4): CRISP
+# at alpha 1.0 / 1.25 / 1.5 against FlexPrefill (JSD routing, gamma-cumsum VS
+# index) at gamma 0.95 / 0.97, plus the first ablation (C_struct routing with
+# the gamma VS index, Table 5's Abl.1).
+COMPARE_METHODS = {
+    "crisp_alpha1.0": dict(router="cstruct", vs_rule="alpha", alpha=1.0, gamma=0.95),
+    "crisp_alpha1.25": dict(router="cstruct", vs_rule="alpha", alpha=1.25, gamma=0.95),
+    "crisp_alpha1.5": dict(router="cstruct", vs_rule="alpha", alpha=1.5, gamma=0.95),
+    "flexprefill_gamma0.95": dict(router="jsd", vs_rule="gamma", alpha=1.0, gamma=0.95),
+    "flexprefill_gamma0.97": dict(router="jsd", vs_rule="gamma", alpha=1.0, gamma=0.97),
+    "abl1_cstruct_gamma0.95": dict(router="cstruct", vs_rule="gamma", alpha=1.0, gamma=0.95),
+}
+
+
+def run_compare(args, out_path):
+    """CRISP vs FlexPrefill on the named workloads: per method the stage
+    times, density, speedup over the dense kernel (timed once per workload)
+    and the routes' agreement with C_struct routing. One JSON line each."""
+    import torch
+    import dynamic_block_sparse_qk_b200 as C
+    from synthetic import WORKLOADS, make_qkv
+
+    dev = torch.device("cuda", 0)
+    timed = _event_timer(dev, max(1, args.steps))
+    for name in args.compare_workloads.split(","):
+        w = WORKLOADS[name].with_(seed=args.seed)
+        q, k, v, _ = make_qkv(w, device=str(dev))
+        base = C.params_for(q, k, block=w.block)
+        ws = C.alloc_workspace(base, dev)
+        dense_ms = timed(lambda: C.crisp_dense_prefill(base, q, k, v, ws, want_lse=False))
+        ref_pattern = None
+        for meth, kw in COMPARE_METHODS.items():
+            p = C.params_for(q, k, block=w.block, **kw)
+            pt = time_point(C, p, q, k, v, ws, timed, dev)
+            pat = pt.pop("_pattern")
+            if ref_pattern is None:
+                ref_pattern = pat
+            rec = {"workload": w.name, "method": meth, **kw, **pt, "dense_ms": round(dense_ms, 4),
+                   "speedup_vs_dense": round(dense_ms / pt["total_ms"], 3),
+                   "speedup_attend_only": round(dense_ms / pt["attend_ms"], 3),
+                   "route_agreement_with_cstruct": round(float((pat == ref_pattern).float().mean()), 4)}
+            with open(out_path, "a") as fo:
+                fo.write(json.dumps(rec) + "\n")
+            print(json.dumps(rec), flush=True)
+        del q, k, v, ws
+        torch.cuda.empty_cache()
+
+
 SWEEP_N = (8192, 16384, 32768, 65536, 131072, 262144, 524288)
 SWEEP_F = (0.0, 0.25, 0.5)
 SWEEP_ALPHA = (0.5, 1.0, 2.0)
@@ -348,19 +450,7 @@ def run_sweep(args, out_path):
                 except (ValueError, KeyError):
                     pass
     dev = torch.device("cuda", 0)
-    stream = torch.cuda.current_stream(dev)
-    reps = max(1, args.steps)
-
-    def timed(fn):
-        fn()
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
-            fn()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        return e0.elapsed_time(e1) / reps
+    timed = _event_timer(dev, max(1, args.steps))
 
     ns = tuple(int(x) for x in args.sweep_n.split(",")) if args.sweep_n else SWEEP_N
     fs = tuple(float(x) for x in args.sweep_f.split(",")) if args.sweep_f else SWEEP_F
@@ -379,37 +469,12 @@ def run_sweep(args, out_path):
             pat_j = C.crisp_route(pj, q, k, ws)[0].clone()
             for a in todo:
                 p = C.params_for(q, k, block=w.block, alpha=a, vs_rule=args.vs_rule)
-                out = {}
-
-                def route():
-                    out["r"] = C.crisp_route(p, q, k, ws)
-
-                def select():
-                    r = out["r"]
-                    out["s"] = C.crisp_select(p, q, k, r[0], r[2], r[3], ws, want_mask=False)
-
-                def attend():
-                    s = out["s"]
-                    out["a"] = C.crisp_sparse_prefill(p, q, k, v, s[1], s[2], ws, want_lse=False)
-
-                with ClockSampler(dev.index if dev.index is not None else 0) as clk:
-                    t_route = timed(route)
-                    t_select = timed(select)
-                    t_attend = timed(attend)
-                pattern, tcnt = out["r"][0], out["s"][2]
-                nb = w.n_blocks
-                causal = p.batch * p.h_q * nb * (nb + 1) // 2
-                total = t_route + t_select + t_attend
+                pt = time_point(C, p, q, k, v, ws, timed, dev)
+                pat = pt.pop("_pattern")
                 rec = {"seq_len": n, "diffuse_frac": f, "alpha": a, "vs_rule": args.vs_rule, "workload": w.name,
-                       "route_ms": round(t_route, 4), "select_ms": round(t_select, 4),
-                       "attend_ms": round(t_attend, 4), "total_ms": round(total, 4),
-                       "dense_ms": round(dense_ms, 4), "speedup_vs_dense": round(dense_ms / total, 3),
-                       "density": round(int(tcnt.sum()) / causal, 5),
-                       "vs_heads": int((pattern == 0).sum()), "heads": p.batch * p.h_q,
-                       "cstruct_jsd_agreement": round(float((pattern == pat_j).float().mean()), 4),
-                       "attend_tflops": round(int(tcnt.sum()) * 4 * w.block ** 2 * w.head_dim
-                                              / (t_attend * 1e-3) / 1e12, 1),
-                       "clocks": clk.summary()}
+                       **pt, "dense_ms": round(dense_ms, 4),
+                       "speedup_vs_dense": round(dense_ms / pt["total_ms"], 3),
+                       "cstruct_jsd_agreement": round(float((pat == pat_j).float().mean()), 4)}
                 with open(out_path, "a") as fo:
                     fo.write(json.dumps(rec) + "\n")
                 print(json.dumps(rec), flush=True)
@@ -531,9 +596,16 @@ def main():
     ap.add_argument("--sweep-n", default=None, help="comma-separated sequence lengths (default: all)")
     ap.add_argument("--sweep-f", default=None, help="comma-separated diffuse-head fractions (default: all)")
     ap.add_argument("--sweep-alpha", default=None, help="comma-separated alpha values (default: 0.5,1,2)")
+    ap.add_argument("--compare", default=None,
+                    help="write the CRISP vs FlexPrefill latency comparison to this JSONL file")
+    ap.add_argument("--compare-workloads", default="qwen_131k,llama_512k",
+                    help="comma-separated workloads of the comparison")
     args = ap.parse_args()
     if args.sweep:
         run_sweep(args, args.sweep)
+        return
+    if args.compare:
+        run_compare(args, args.compare)
         return
 
     rank = int(os.environ.get("RANK", "0"))

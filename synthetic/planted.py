@@ -82,7 +82,14 @@ WORKLOADS: Dict[str, Workload] = {
                      n_vertical=0, recency_peak=9.0, recency_freqs="rope"),
     "llama_32k": Workload("llama_32k", 1, 32, 8, 128, 32768, 128),
     "qwen_131k": Workload("qwen_131k", 1, 28, 4, 128, 131072, 128, sink_logit_range=(1.0, 6.0)),
+    "llama_128k": Workload("llama_128k", 1, 32, 8, 128, 131072, 128),
     "llama_512k": Workload("llama_512k", 1, 32, 8, 128, 524288, 128),
+    # the same shapes with a decaying RoPE-style recency band (geometric
+    # frequencies 10000**(-k/8), peak logit 9) instead of the block-periodic one
+    "llama_32k_rope": Workload("llama_32k_rope", 1, 32, 8, 128, 32768, 128, recency_peak=9.0,
+                               recency_freqs="rope"),
+    "llama_512k_rope": Workload("llama_512k_rope", 1, 32, 8, 128, 524288, 128, recency_peak=9.0,
+                                recency_freqs="rope"),
     # four prompts of different lengths (none a multiple of the block but the
     # first) in one padded batch
     "llama_varlen_131k": Workload("llama_varlen_131k", 4, 32, 8, 128, 131072, 128,
