@@ -28,7 +28,7 @@ PATTERN_VS, PATTERN_PE = 0, 1
 EXPORTED = ("crisp_version", "crisp_status_string", "crisp_check_params", "crisp_workspace_size",
             "crisp_route", "crisp_select", "crisp_sparse_prefill", "crisp_dense_prefill",
             "crisp_get_device_status", "crisp_route_noalloc", "crisp_selftest_wait_timeout",
-            "crisp_selftest_pipeline_timeout")
+            "crisp_selftest_pipeline_timeout", "crisp_prefill_host_workspace_size", "crisp_prefill_host")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -111,6 +111,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.crisp_selftest_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
     lib.crisp_selftest_pipeline_timeout.restype = i32
     lib.crisp_selftest_pipeline_timeout.argtypes = [P, vp, vp, vp, vp, vp, sz, ctypes.c_longlong, vp]
+    lib.crisp_prefill_host_workspace_size.restype = sz
+    lib.crisp_prefill_host_workspace_size.argtypes = [P, i32]
+    lib.crisp_prefill_host.restype = i32
+    lib.crisp_prefill_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]
     lib.crisp_get_device_status.restype = i32
     lib.crisp_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), vp]
     _lib = lib
@@ -274,3 +278,26 @@ def crisp_selftest_pipeline_timeout(p: CrispParams, q, k, v, o, ws, limit_cycles
     _check("crisp_selftest_pipeline_timeout", load_library().crisp_selftest_pipeline_timeout(
         ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(ws), ws.numel(), int(limit_cycles),
         _stream(stream)))
+
+
+def crisp_prefill_host_workspace_size(p: CrispParams, kv_per_chunk: int = 1) -> int:
+    n = load_library().crisp_prefill_host_workspace_size(ctypes.byref(p), int(kv_per_chunk))
+    if n == 0:
+        _check("crisp_prefill_host_workspace_size", load_library().crisp_check_params(ctypes.byref(p)))
+        raise CrispError("crisp_prefill_host_workspace_size", -1)
+    return int(n)
+
+
+def crisp_prefill_host(p: CrispParams, q, k, v, o, ws, lse=None, seq_lens=None, pattern=None,
+                       kv_per_chunk: int = 1, stream=None) -> None:
+    """The whole prefill on pinned host tensors (see include/crisp.h):
+    synchronous; ``seq_lens`` a host int32 tensor or None, ``pattern`` an
+    optional host int32 tensor [batch * h_q] receiving the routes, ``ws`` a
+    device uint8 tensor of crisp_prefill_host_workspace_size bytes."""
+    _need_cuda(ws)
+    for t in (q, k, v, o, lse, seq_lens, pattern):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError("crisp_prefill_host takes contiguous host tensors")
+    _check("crisp_prefill_host", load_library().crisp_prefill_host(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(seq_lens), _ptr(pattern),
+        int(kv_per_chunk), _ptr(ws), ws.numel(), _stream(stream)))

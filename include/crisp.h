@@ -168,6 +168,38 @@ int crisp_sparse_prefill(const crisp_params* p, const void* q, const void* k, co
 int crisp_dense_prefill(const crisp_params* p, const void* q, const void* k, const void* v,
                         void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
 
+/* Device workspace bytes crisp_prefill_host needs for `p` with
+ * `kv_per_chunk` KV heads per chunk (0 when the arguments are invalid). */
+size_t crisp_prefill_host_workspace_size(const crisp_params* p, int kv_per_chunk);
+
+/* Algorithm 1 end to end on HOST buffers: route (Algorithm 2), select
+ * (Algorithms 3, 4, 6) and block-sparse attention (Eq. 1), exactly as
+ * crisp_route + crisp_select + crisp_sparse_prefill, for inputs and outputs
+ * in page-locked host memory (cudaHostAlloc / cudaMallocHost or
+ * cudaHostRegister over the whole array).
+ *  - q, k, v: host bf16 [batch][heads][seqlen][head_dim]; o: host bf16
+ *    [batch][h_q][seqlen][head_dim]; lse (may be NULL): host float32
+ *    [batch][h_q][seqlen]. Only the first seq_lens[b] rows of sequence b are
+ *    read and written; other rows of o and lse keep their contents.
+ *  - seq_lens (may be NULL = all seqlen): HOST int32 [batch], each in
+ *    (2*block, seqlen] (else CRISP_ERR_SHAPE). p->seq_lens must be NULL.
+ *  - pattern (may be NULL): host int32 [batch * h_q] receiving the routes.
+ *  - The prefill runs in chunks of one sequence and kv_per_chunk KV heads
+ *    (a divisor of h_kv) with their query heads. Two slots of device
+ *    buffers in `ws` (caller-owned device memory, 256-byte aligned, at least
+ *    crisp_prefill_host_workspace_size bytes) alternate between chunks: the
+ *    host-to-device copies of chunk i+1 and the device-to-host copies of
+ *    chunk i-1 overlap the kernels of chunk i (one cudaMemcpy2DAsync per
+ *    tensor and chunk). The kernels run on `stream`, after the work already
+ *    queued there; the copies on two streams the call creates and destroys.
+ *  - The call is synchronous: it returns once o (and lse, pattern) hold the
+ *    result. Kernel-side errors of any chunk are returned directly
+ *    (CRISP_ERR_TIMEOUT, CRISP_ERR_DEVICE); pageable host pointers return
+ *    CRISP_ERR_ARG before any copy. The library allocates no device memory. */
+int crisp_prefill_host(const crisp_params* p, const void* q, const void* k, const void* v, void* o,
+                       float* lse, const int32_t* seq_lens, int32_t* pattern, int kv_per_chunk,
+                       void* ws, size_t ws_bytes, void* stream);
+
 /* Routing without a caller workspace. The paper has no counterpart: this
  * entry point exists for callers that may not allocate device memory — for
  * example a plug-in whose host framework reserves all device memory for its

@@ -19,9 +19,26 @@ ATTN_MAX_ABS = 2e-2
 ATTN_MEAN_ABS = 2e-3
 
 
+def lists_match_mask_on_device(mask, tile_idx, tile_cnt):
+    """Tile lists must hold, per query block, the ascending key blocks of its
+    mask row: checked with torch on the device, one head at a time (at 512k
+    the lists are 2 GiB, too large to bring to the host for every config)."""
+    nb = mask.shape[-1]
+    cols = torch.arange(nb, device=mask.device, dtype=torch.int32)
+    for bh in range(mask.shape[0]):
+        m = mask[bh].bool()
+        assert torch.equal(m.sum(-1, dtype=torch.int32), tile_cnt[bh]), bh
+        pos = (torch.cumsum(m.to(torch.int32), dim=-1) - 1).clamp_(min=0).long()
+        got = torch.gather(tile_idx[bh], -1, pos)
+        assert torch.equal(got[m], cols.expand(nb, nb)[m]), bh
+
+
 def run_gpu(w, q, k, v, router="cstruct", vs_rule="alpha", alpha=1.0, gamma=0.95, tau_jsd=0.1,
-            granularity="tile"):
-    """Runs route -> select -> sparse prefill through the C ABI; returns CPU copies."""
+            granularity="tile", keep_on_device=False):
+    """Runs route -> select -> sparse prefill through the C ABI; returns CPU
+    copies. With keep_on_device the tile lists are checked against the mask
+    on the device and dropped, and o / lse stay on the device (compare_head
+    then brings only the compared rows to the host)."""
     import dynamic_block_sparse_qk_b200 as C
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     lens = None if w.lengths is None else torch.tensor(list(w.lengths), dtype=torch.int32, device=qd.device)
@@ -36,7 +53,16 @@ def run_gpu(w, q, k, v, router="cstruct", vs_rule="alpha", alpha=1.0, gamma=0.95
     status = C.crisp_get_device_status(ws)
     out = {"pattern": pattern, "score": score, "p_v": p_v, "p_s": p_s, "vs_sel": vs_sel,
            "mask": mask, "tile_idx": tidx, "tile_cnt": tcnt, "o": o, "lse": lse}
-    out = {key: val.cpu() for key, val in out.items()}
+    if keep_on_device:
+        assert granularity == "tile"
+        lists_match_mask_on_device(mask, tidx, tcnt)
+        dev = {"o": o, "lse": lse}
+        out = {key: val.cpu() for key, val in out.items() if key not in ("o", "lse", "tile_idx")}
+        out.update(dev)
+        out["lists_checked"] = True
+        del tidx
+    else:
+        out = {key: val.cpu() for key, val in out.items()}
     out["status"] = status
     out["params"] = p
     del qd, kd, vd, ws, lens
@@ -126,13 +152,35 @@ def pe_exempt(a_bar: np.ndarray, gamma: float) -> np.ndarray:
     return ex
 
 
-def compare_head(gpu, b, h, q_head, k_head, v_head, w, oprm, qblocks=None, score_tol=2e-5):
-    """Compares one query head; returns a report dict (asserts on hard failures)."""
+def oracle_for_alphas(q_head, k_head, oprms):
+    """Oracle results for parameter sets that differ only in alpha: routing
+    and the PE index (which alpha does not enter) once, then the VS index of
+    Algorithm 3 and its tile mask per alpha, with the same oracle functions
+    head_route_and_select composes."""
+    base = O.head_route_and_select(q_head, k_head, oprms[0])
+    outs = [base]
+    n = q_head.shape[0]
+    for prm in oprms[1:]:
+        assert prm.vs_rule in ("alpha", "alpha_median") and prm.block == oprms[0].block
+        r = dict(base)
+        if base["pattern"] == O.VS:
+            floor = "median" if prm.vs_rule == "alpha_median" else "mean"
+            r["s_v"] = O.vs_index_alpha(base["p_v"], prm.alpha, prm.k_min_blocks, floor)
+            r["s_s"] = O.vs_index_alpha(base["p_s"], prm.alpha, prm.k_min_blocks, floor)
+            r["mask"] = O.vs_tile_mask(r["s_v"], r["s_s"], O.n_blocks(n, prm.block), n, prm.block)
+        outs.append(r)
+    return outs
+
+
+def compare_head(gpu, b, h, q_head, k_head, v_head, w, oprm, qblocks=None, score_tol=2e-5, orc=None):
+    """Compares one query head; returns a report dict (asserts on hard failures).
+    ``orc``: the oracle's result for this head and oprm when already computed."""
     bh = b * w.h_q + h
     n = q_head.shape[0]                        # this sequence's length
     nb = O.n_blocks(n, w.block)                # its blocks; GPU arrays are w.n_blocks wide
     rep = {"head": (b, h), "exempt_route": False, "exempt_blocks": 0}
-    orc = O.head_route_and_select(q_head, k_head, oprm)
+    if orc is None:
+        orc = O.head_route_and_select(q_head, k_head, oprm)
     gp = int(gpu["pattern"][bh])
     # (1) block scores (zero past the sequence's own blocks)
     for key in ("p_v", "p_s"):
@@ -181,12 +229,12 @@ def compare_head(gpu, b, h, q_head, k_head, v_head, w, oprm, qblocks=None, score
     assert not cnt_full[nb:].any()
     cnt = cnt_full[:nb]
     np.testing.assert_array_equal(cnt, gmask.sum(axis=1))
-    tidx = gpu["tile_idx"][bh].numpy()
     token = oprm.granularity == "token"
     vs_tokens = None
     if token and gp == O.VS:
         vs_tokens = (np.nonzero(sel[0])[0], np.nonzero(sel[1])[0])
-    for qb in range(nb):
+    tidx = None if gpu.get("lists_checked") else gpu["tile_idx"][bh].numpy()
+    for qb in (range(nb) if tidx is not None else ()):
         ids = tidx[qb, : cnt[qb]]
         if token:
             flags = ids & ~TILE_ID_MASK
@@ -196,14 +244,15 @@ def compare_head(gpu, b, h, q_head, k_head, v_head, w, oprm, qblocks=None, score
             np.testing.assert_array_equal(flags, want)
         np.testing.assert_array_equal(ids, np.nonzero(gmask[qb])[0])
     rep["density"] = float(gmask.sum()) / (nb * (nb + 1) / 2)
+    rep["qblocks"] = nb if qblocks is None else len(qblocks)
     # (5) attention on the GPU's own mask
     o_ref, lse_ref, rows = O.masked_attention_rows(q_head, k_head, v_head, gmask, w.block,
                                                    oprm.scale(q_head.shape[1]), qblocks, vs_tokens)
-    o_all = gpu["o"][b, h].float().numpy()
-    lse_all = gpu["lse"][b, h].numpy()
-    assert not o_all[n:].any() and np.all(lse_all[n:] == -np.inf)     # padding rows
-    o_gpu = o_all[rows]
-    lse_gpu = lse_all[rows]
+    o_all, lse_all = gpu["o"][b, h], gpu["lse"][b, h]            # host or device tensors
+    assert not o_all[n:].any() and bool(torch.all(lse_all[n:] == -float("inf")))     # padding rows
+    sel_rows = torch.as_tensor(rows, dtype=torch.long, device=o_all.device)
+    o_gpu = o_all[sel_rows].float().cpu().numpy()
+    lse_gpu = lse_all[sel_rows].cpu().numpy()
     err = np.abs(o_gpu - o_ref)
     rep["attn_max_abs"] = float(err.max())
     rep["attn_mean_abs"] = float(err.mean())
@@ -218,6 +267,28 @@ def sample_qblocks(nb: int, n_random: int, seed: int) -> Sequence[int]:
     pick = {0, nb - 1}
     pick.update(int(x) for x in rng.choice(np.arange(1, nb - 1), size=min(n_random, nb - 2), replace=False))
     return sorted(pick)
+
+
+# Per-case parity summaries of this pytest session (printed at its end by
+# the terminal-summary hook in conftest.py): how many routing decisions and
+# selected blocks were excused under the 1e-4 exemption rule, and the
+# attention errors.
+SESSION_REPORTS = []
+
+
+def record(case: str, reps, **extra) -> dict:
+    """Adds one parity case's summary to SESSION_REPORTS and returns it."""
+    rec = {"case": case, "heads": len(reps),
+           "vs_heads": sum(1 for r in reps if r.get("pattern") == O.VS),
+           "exempt_routes": sum(int(r["exempt_route"]) for r in reps),
+           "exempt_blocks": sum(int(r["exempt_blocks"]) for r in reps),
+           "qblocks_compared": sum(int(r.get("qblocks", 0)) for r in reps),
+           "attn_max_abs": max((r["attn_max_abs"] for r in reps), default=0.0),
+           "attn_mean_abs": max((r["attn_mean_abs"] for r in reps), default=0.0),
+           "density": (sum(r["density"] for r in reps) / len(reps)) if reps else 0.0}
+    rec.update(extra)
+    SESSION_REPORTS.append(rec)
+    return rec
 
 
 def compare_all(w, q, k, v, gpu, oprm, qblocks_fn=None, heads=None):

@@ -102,6 +102,26 @@ def test_entry_points_validate_before_launch(lib):
                                                None) == -3
 
 
+def test_host_prefill_validates_before_any_copy(lib):
+    p = _p(seqlen=4096)
+    fake = ctypes.c_void_p(1 << 20)
+    need = lib.crisp_prefill_host_workspace_size(ctypes.byref(p), 1)
+    assert need > 0
+    assert lib.crisp_prefill_host_workspace_size(ctypes.byref(p), 3) == 0        # 3 does not divide h_kv = 8
+    assert lib.crisp_prefill_host_workspace_size(ctypes.byref(p), 0) == 0
+    assert lib.crisp_prefill_host_workspace_size(ctypes.byref(p), 2) > need     # bigger chunks, bigger slots
+    assert lib.crisp_prefill_host(ctypes.byref(p), None, fake, fake, fake, None, None, None, 1, fake, need,
+                                  None) == -1
+    assert lib.crisp_prefill_host(ctypes.byref(p), fake, fake, fake, fake, None, None, None, 1, fake, need - 1,
+                                  None) == -3
+    assert lib.crisp_prefill_host(ctypes.byref(p), fake, fake, fake, fake, None, None, None, 1,
+                                  ctypes.c_void_p((1 << 20) + 8), need, None) == -1
+    withlens = _p(seqlen=4096)
+    withlens.seq_lens = ctypes.c_void_p(1 << 20)                # device lengths are not taken here
+    assert lib.crisp_prefill_host(ctypes.byref(withlens), fake, fake, fake, fake, None, None, None, 1, fake,
+                                  need, None) == -1
+
+
 def test_selftest_validates_before_launch(lib):
     fake = ctypes.c_void_p(1 << 20)                       # aligned, never dereferenced on failure
     assert lib.crisp_selftest_wait_timeout(None, 1000, None) == -1
@@ -181,8 +201,8 @@ int main(void) {
 
 
 def test_host_input_prefill_rejects_unpinned_tensors():
-    # prefill_from_host copies asynchronously from page-locked memory only; a
-    # pageable (or device) tensor is refused before any stream or copy exists
+    # prefill_from_host copies from page-locked memory only; a pageable (or
+    # device) tensor is refused before any stream, workspace or copy exists
     import torch
     from dynamic_block_sparse_qk_b200 import prefill_from_host
     q = torch.zeros(1, 4, 1024, 64, dtype=torch.bfloat16)

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import oracle as O
-from synthetic import WORKLOADS, Workload, make_qkv
+from synthetic import WORKLOADS, Workload, make_qkv, sweep_workload
 import parity_util as PU
 
 pytestmark = pytest.mark.gpu
@@ -25,17 +25,58 @@ def _lib():
 
 
 def _check(w, router="cstruct", vs_rule="alpha", alpha=1.0, gamma=0.95, qblocks_fn=None,
-           heads=None, expect_both=False, granularity="tile"):
-    q, k, v, meta = make_qkv(w)
+           heads=None, expect_both=False, granularity="tile", inputs=None, keep_on_device=False):
+    q, k, v, meta = make_qkv(w) if inputs is None else inputs
     gpu = PU.run_gpu(w, q, k, v, router=router, vs_rule=vs_rule, alpha=alpha, gamma=gamma,
-                     granularity=granularity)
+                     granularity=granularity, keep_on_device=keep_on_device)
     assert gpu["status"] == 0
     oprm = PU.oracle_params(w, router=router, vs_rule=vs_rule, alpha=alpha, gamma=gamma,
                             granularity=granularity)
     reps = PU.compare_all(w, q, k, v, gpu, oprm, qblocks_fn=qblocks_fn, heads=heads)
+    PU.record(f"{w.name} {router} {vs_rule} alpha={alpha} gamma={gamma} {granularity}", reps)
     if expect_both:
         pats = {r["pattern"] for r in reps}
         assert pats == {O.VS, O.PE}, pats
+    return reps
+
+
+def _device_inputs(w):
+    """Inputs generated on the GPU (fast at 64k-512k), copied to the host for
+    the oracle; the CUDA path receives the same values."""
+    q, k, v, meta = make_qkv(w, device="cuda")
+    out = (q.cpu(), k.cpu(), v.cpu(), meta)
+    del q, k, v
+    torch.cuda.empty_cache()
+    return out
+
+
+def _check_alphas(w, alphas, qblocks_fn, inputs, expect_both=False):
+    """One input, several alpha values: each alpha is a full GPU prefill
+    (route, select, attention) compared with the oracle; the oracle routes and
+    runs the PE index once per head and the VS index once per alpha."""
+    q, k, v, _ = inputs
+    oprms = [PU.oracle_params(w, alpha=a) for a in alphas]
+    gpus = []
+    for a in alphas:
+        gpu = PU.run_gpu(w, q, k, v, alpha=a, keep_on_device=True)
+        assert gpu["status"] == 0
+        gpus.append(gpu)
+    g = w.h_q // w.h_kv
+    reps = [[] for _ in alphas]
+    kv_cache = {}
+    for h in range(w.h_q):
+        if h // g not in kv_cache:
+            kv_cache = {h // g: (O.bf16_to_f64(k[0, h // g]), O.bf16_to_f64(v[0, h // g]))}
+        kh, vh = kv_cache[h // g]
+        qh = O.bf16_to_f64(q[0, h])
+        orcs = PU.oracle_for_alphas(qh, kh, oprms)
+        for i in range(len(alphas)):
+            reps[i].append(PU.compare_head(gpus[i], 0, h, qh, kh, vh, w, oprms[i], qblocks_fn(i, h),
+                                           orc=orcs[i]))
+    for i, a in enumerate(alphas):
+        PU.record(f"{w.name} cstruct alpha alpha={a} gamma=0.95 tile", reps[i])
+        if expect_both:
+            assert {r["pattern"] for r in reps[i]} == {O.VS, O.PE}
     return reps
 
 
@@ -275,14 +316,44 @@ def test_variable_length_llama_32k():
     assert {r["pattern"] for r in reps} == {O.VS, O.PE}
 
 
+# ---- the large configurations: routing and selection of every head in full;
+# attention on the first, the last and 30 random query blocks of every head
+def _sample32(nb, base):
+    return lambda b, h: PU.sample_qblocks(nb, 30, base + h)
+
+
 @pytest.mark.slow
 def test_qwen_131k_alpha_and_gamma():
     w = WORKLOADS["qwen_131k"]
+    inputs = _device_inputs(w)
     for vs_rule in ("alpha", "gamma"):
-        _check(w, vs_rule=vs_rule, qblocks_fn=lambda b, h: PU.sample_qblocks(w.n_blocks, 2, 2000 + h))
+        _check(w, vs_rule=vs_rule, qblocks_fn=_sample32(w.n_blocks, 2000), inputs=inputs, keep_on_device=True)
 
 
 @pytest.mark.slow
-def test_llama_512k():
+def test_llama_512k_alpha_schedule():
+    # the headline input at alpha 1 (30 random query blocks per head) and the
+    # CRISP page's speed settings alpha 1.25 and 1.5 (Section 5.3; 2 random)
     w = WORKLOADS["llama_512k"]
-    _check(w, qblocks_fn=lambda b, h: PU.sample_qblocks(w.n_blocks, 1, 3000 + h), expect_both=True)
+    nb = w.n_blocks
+    reps = _check_alphas(w, (1.0, 1.25, 1.5), lambda i, h: PU.sample_qblocks(nb, 30 if i == 0 else 2, 3000 + h),
+                         _device_inputs(w), expect_both=True)
+    assert sum(r["pattern"] == O.VS for r in reps[0]) == 24
+
+
+# ---- sweep points beyond alpha = 1: selection in full, attention sampled
+@pytest.mark.slow
+@pytest.mark.parametrize("seqlen,f", [(65536, 0.0), (65536, 0.5), (524288, 0.0), (524288, 0.5)])
+def test_sweep_points_alpha_half_and_two(seqlen, f):
+    w = sweep_workload(seqlen, f)
+    nb = w.n_blocks
+    n_random = 4 if seqlen <= 65536 else 1
+    _check_alphas(w, (0.5, 2.0), lambda i, h: PU.sample_qblocks(nb, n_random, 6000 + 31 * i + h),
+                  _device_inputs(w), expect_both=f > 0)
+
+
+# ---- a workload with a RoPE-style recency band (geometric frequencies)
+def test_llama_32k_rope_recency():
+    w = WORKLOADS["llama_32k_rope"]
+    reps = _check(w, qblocks_fn=lambda b, h: PU.sample_qblocks(w.n_blocks, 4, 7000 + h), expect_both=True)
+    assert sum(r["pattern"] == O.VS for r in reps) == 24
