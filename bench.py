@@ -114,6 +114,32 @@ def max_over_ranks(values, device):
     return [float(x) for x in t.tolist()]
 
 
+def sum_over_ranks(values, device):
+    """Element-wise sum of a list of numbers over all ranks (identity when
+    not distributed): the whole job's tiles and heads under head sharding."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(x) for x in values]
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t.tolist()]
+
+
+def rank_problem(w, args, rank, world):
+    """The workload this rank runs and the KV heads it owns: with --shard
+    replicas every rank runs its own whole problem (seed + rank); with
+    --shard heads rank r runs KV heads kv_head_range(H_kv, N, r) of one
+    problem with their query heads (same seed on every rank)."""
+    from dynamic_block_sparse_qk_b200.shard import kv_head_range
+    if args.shard == "heads":
+        kv = kv_head_range(w.h_kv, world, rank)
+        g = w.h_q // w.h_kv
+        return w.with_(seed=args.seed), list(kv), w.with_(h_q=len(kv) * g, h_kv=len(kv))
+    wr = w.with_(seed=args.seed + rank)
+    return wr, None, wr
+
+
 def launches_per_step(router: str) -> dict:
     """Kernels of this library launched by one call of each stage."""
     route = 2 + (2 if router == "jsd" else 0)      # proxy stats (+ merge), scores (+ C_struct route),
@@ -169,8 +195,8 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = WORKLOADS[args.workload].with_(seed=args.seed + rank)
-    q, k, v, meta = make_qkv(w, device=str(dev))
+    w_full, kv_heads, w = rank_problem(WORKLOADS[args.workload], args, rank, world)
+    q, k, v, meta = make_qkv(w_full, device=str(dev), heads_kv=kv_heads)
     lens = None if w.lengths is None else torch.tensor(list(w.lengths), dtype=torch.int32, device=dev)
     p = C.params_for(q, k, block=w.block, alpha=args.alpha, gamma=args.gamma, router=args.router,
                      vs_rule=args.vs_rule, seq_lens=lens, granularity=args.granularity)
@@ -243,7 +269,14 @@ def run_ours(args, rank, world, local_rank):
     dense_ms = statistics.mean(dts) if dts else float("nan")
     del od
 
-    ms, dense_ms = max_over_ranks([ms_local, dense_ms], dev)
+    ms, dense_ms, attend_ms = max_over_ranks([ms_local, dense_ms, stages["attend"]], dev)
+    if args.shard == "heads":
+        # the job's work is the sum of the ranks' slices; its time the slowest rank's
+        cnt_sum, causal_tiles, n_vs, bh_all = (int(x) for x in sum_over_ranks(
+            [cnt_sum, causal_tiles, n_vs, p.batch * p.h_q], dev))
+        stages["attend"] = attend_ms
+    else:
+        bh_all = p.batch * p.h_q
 
     # end-to-end through the public API with host buffers (H2D inputs, D2H output)
     e2e = None
@@ -296,8 +329,10 @@ def run_ours(args, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": round(ms, 3), "unit": "ms", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {**workload_config(w, args), "parallelism": f"replicas{world}",
+        "scaling": "strong" if args.shard == "heads" else "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {**workload_config(w_full, args),
+                   "parallelism": f"{'kv_heads' if args.shard == 'heads' else 'replicas'}{world}",
                    "l2": "flushed between steps" if flush is not None else
                          f"inputs ({in_bytes / 2**30:.1f} GiB) larger than L2"},
         "stages_ms": {k_: round(v_, 3) for k_, v_ in stages.items()},
@@ -305,7 +340,7 @@ def run_ours(args, rank, world, local_rank):
         "speedup_vs_dense": round(dense_ms / ms, 3),
         "speedup_attend_only": round(dense_ms / stages["attend"], 3),
         "route_select_frac": round((stages["route"] + stages["select"]) / ms, 4),
-        "density": round(cnt_sum / causal_tiles, 5), "vs_heads": n_vs, "heads": bh,
+        "density": round(cnt_sum / causal_tiles, 5), "vs_heads": n_vs, "heads": bh_all,
         "executed_tiles": cnt_sum,
         "attend_tflops": round(attn_tflops, 1), "dense_tflops": round(dense_tflops, 1),
         "roofline": {"bound": "tensor", "kernel": "attention (sparse)", "achieved": round(attn_tflops, 1),
@@ -593,6 +628,9 @@ def main():
     ap.add_argument("--granularity", default="tile", choices=["tile", "token"],
                     help="VS mask: selected blocks as whole tiles, or slash blocks as diagonal bands")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="N > 1: independent replicas per rank (weak scaling), or one problem split by "
+                         "KV-head groups (strong scaling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=20.0)

@@ -150,18 +150,27 @@ def _rope_block(w: Workload, pos: torch.Tensor, amp: float) -> torch.Tensor:
     return out.to(torch.float32)
 
 
-def make_qkv(w: Workload, device: str = "cpu", heads_q: Optional[Sequence[int]] = None):
+def make_qkv(w: Workload, device: str = "cpu", heads_q: Optional[Sequence[int]] = None,
+             heads_kv: Optional[Sequence[int]] = None):
     """Return (q, k, v, meta) as bf16 tensors [B, H, N, d] on ``device``.
 
     ``heads_q`` restricts generation to a subset of query heads (their KV
     heads are generated in full); the returned q then holds only those heads.
+    ``heads_kv`` restricts k and v to those KV heads and, unless heads_q is
+    given, q to their query heads: a slice of the whole problem, with the
+    same values the whole generation gives those heads (every slice has its
+    own seeded generator).
     """
     d, N = w.head_dim, w.seqlen
     c4 = d ** 0.25
     meta = head_kinds(w)
     diffuse = set(meta["diffuse"])
     g = w.h_q // w.h_kv
-    hq_list = list(range(w.h_q)) if heads_q is None else list(heads_q)
+    hk_list = list(range(w.h_kv)) if heads_kv is None else list(heads_kv)
+    if heads_q is not None:
+        hq_list = list(heads_q)
+    else:
+        hq_list = [hk * g + i for hk in hk_list for i in range(g)]
     rec_amp = math.sqrt(w.recency_peak / 8.0) * c4
     pos = torch.arange(N, device=device)
     rope = _rope_block(w, pos, rec_amp) if w.recency_peak > 0 else None
@@ -173,8 +182,8 @@ def make_qkv(w: Workload, device: str = "cpu", heads_q: Optional[Sequence[int]] 
 
     inv = 1.0 / math.sqrt(d)
     q = torch.empty((w.batch, len(hq_list), N, d), dtype=torch.bfloat16, device=device)
-    k = torch.empty((w.batch, w.h_kv, N, d), dtype=torch.bfloat16, device=device)
-    v = torch.empty((w.batch, w.h_kv, N, d), dtype=torch.bfloat16, device=device)
+    k = torch.empty((w.batch, len(hk_list), N, d), dtype=torch.bfloat16, device=device)
+    v = torch.empty((w.batch, len(hk_list), N, d), dtype=torch.bfloat16, device=device)
 
     def pad(x: torch.Tensor, tag: int, b: int, h: int) -> torch.Tensor:
         n_b = w.length(b)
@@ -184,7 +193,7 @@ def make_qkv(w: Workload, device: str = "cpu", heads_q: Optional[Sequence[int]] 
             x[n_b:] = torch.randn((N - n_b, d), generator=gen, device=device, dtype=torch.float32) * 64.0
         return x
     for b in range(w.batch):
-        for hk in range(w.h_kv):
+        for j, hk in enumerate(hk_list):
             x = randn(1, b, hk).mul_(inv)
             x[:, :N_RESERVED] = 0.0
             x[:N_SINK_ROWS, SINK_DIM] += 4.0 * c4
@@ -192,11 +201,11 @@ def make_qkv(w: Workload, device: str = "cpu", heads_q: Optional[Sequence[int]] 
                 x[p, VERT_DIM] += 3.0 * c4
             if rope is not None:
                 x[:, :16] += rope
-            k[b, hk] = pad(x, 11, b, hk).to(torch.bfloat16)
+            k[b, j] = pad(x, 11, b, hk).to(torch.bfloat16)
             x = randn(2, b, hk)
             if not w.v_unit:
                 x.mul_(inv)
-            v[b, hk] = pad(x, 12, b, hk).to(torch.bfloat16)
+            v[b, j] = pad(x, 12, b, hk).to(torch.bfloat16)
         for i, h in enumerate(hq_list):
             x = randn(0, b, h).mul_(inv)
             if h not in diffuse:

@@ -37,3 +37,17 @@ def test_reference_arm_other_ranks_do_no_work():
     proc = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert proc.returncode == 0, proc.stderr[-2000:]
     assert proc.stdout.strip() == ""
+
+
+def test_rank_problem_replicas_and_kv_head_shards():
+    import argparse
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    from synthetic import WORKLOADS
+    w = WORKLOADS["llama_512k"]
+    full, kv, local = bench.rank_problem(w, argparse.Namespace(shard="heads", seed=0), rank=1, world=4)
+    assert kv == [2, 3] and full.seed == 0 and full.h_q == 32
+    assert (local.h_q, local.h_kv, local.seqlen) == (8, 2, w.seqlen)
+    full, kv, local = bench.rank_problem(w, argparse.Namespace(shard="replicas", seed=0), rank=1, world=4)
+    assert kv is None and full is local and full.seed == 1 and full.h_q == 32
