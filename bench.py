@@ -140,12 +140,15 @@ def rank_problem(w, args, rank, world):
     return wr, None, wr
 
 
-def launches_per_step(router: str) -> dict:
+def launches_per_step(router: str, n_blocks: int) -> dict:
     """Kernels of this library launched by one call of each stage."""
     route = 2 + (2 if router == "jsd" else 0)      # proxy stats (+ merge), scores (+ C_struct route),
     #                                                 JSD only: K pool, JSD route
-    select = 9                                      # vs select, K/Q pool, PE logits/normalise,
-    #                                                 3 x hist (+ cut), tie count (+ scan), tiles
+    if n_blocks * (n_blocks + 1) // 2 <= 256 * 257 // 2:
+        select = 5                                  # vs select, K/Q pool, PE logits, one-CTA PE cut, tiles
+    else:
+        select = 9                                  # vs select, K/Q pool, PE logits/normalise,
+        #                                             3 x hist (+ cut), tie count (+ scan), tiles
     return {"route": route, "select": select, "attention": 1, "total": route + select + 1}
 
 
@@ -355,7 +358,7 @@ def run_ours(args, rank, world, local_rank):
                            "frac_of_hbm": round(v_ / (stages[k_] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
                       for k_, v_ in stage_bytes.items()},
         "e2e": e2e,
-        "gpu_launches": launches_per_step(args.router)["total"] * args.steps,
+        "gpu_launches": launches_per_step(args.router, nb)["total"] * args.steps,
         "device_status": status,
         "clocks": clk.summary(),
     }
@@ -397,17 +400,32 @@ def time_point(C, p, q, k, v, ws, timed, dev) -> dict:
             "device_status": status, "clocks": clk.summary(), "_pattern": pattern.clone()}
 
 
-def _event_timer(dev, reps):
+def _event_timer(dev, reps, graphs=False):
+    """timed(fn): mean CUDA-event time of `reps` runs of fn after one
+    warm-up. With graphs, fn (a sequence of library calls) is captured once
+    into a CUDA graph and the graph is replayed, so the time is the GPU's
+    alone, without the host's per-call overhead (how a serving loop that
+    captures its prefill runs it); the outputs fn stores stay valid."""
     import torch
     stream = torch.cuda.current_stream(dev)
+    keep = []
 
     def timed(fn):
         fn()
         torch.cuda.synchronize(dev)
+        run = fn
+        if graphs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, capture_error_mode="relaxed"):
+                fn()
+            keep.append(g)
+            run = g.replay
+            run()
+            torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(reps):
-            fn()
+            run()
         e1.record(stream)
         torch.cuda.synchronize(dev)
         return e0.elapsed_time(e1) / reps
@@ -437,7 +455,7 @@ def run_compare(args, out_path):
     from synthetic import WORKLOADS, make_qkv
 
     dev = torch.device("cuda", 0)
-    timed = _event_timer(dev, max(1, args.steps))
+    timed = _event_timer(dev, max(1, args.steps), graphs=args.graphs)
     for name in args.compare_workloads.split(","):
         w = WORKLOADS[name].with_(seed=args.seed)
         q, k, v, _ = make_qkv(w, device=str(dev))
@@ -452,6 +470,7 @@ def run_compare(args, out_path):
             if ref_pattern is None:
                 ref_pattern = pat
             rec = {"workload": w.name, "method": meth, **kw, **pt, "dense_ms": round(dense_ms, 4),
+                   "timing": "cuda_graph" if args.graphs else "eager",
                    "speedup_vs_dense": round(dense_ms / pt["total_ms"], 3),
                    "speedup_attend_only": round(dense_ms / pt["attend_ms"], 3),
                    "route_agreement_with_cstruct": round(float((pat == ref_pattern).float().mean()), 4)}
@@ -489,7 +508,7 @@ def run_sweep(args, out_path):
                 except (ValueError, KeyError):
                     pass
     dev = torch.device("cuda", 0)
-    timed = _event_timer(dev, max(1, args.steps))
+    timed = _event_timer(dev, max(1, args.steps), graphs=args.graphs)
 
     ns = tuple(int(x) for x in args.sweep_n.split(",")) if args.sweep_n else SWEEP_N
     fs = tuple(float(x) for x in args.sweep_f.split(",")) if args.sweep_f else SWEEP_F
@@ -511,6 +530,7 @@ def run_sweep(args, out_path):
                 pt = time_point(C, p, q, k, v, ws, timed, dev)
                 pat = pt.pop("_pattern")
                 rec = {"seq_len": n, "diffuse_frac": f, "alpha": a, "vs_rule": args.vs_rule, "workload": w.name,
+                       "timing": "cuda_graph" if args.graphs else "eager",
                        **pt, "dense_ms": round(dense_ms, 4),
                        "speedup_vs_dense": round(dense_ms / pt["total_ms"], 3),
                        "cstruct_jsd_agreement": round(float((pat == pat_j).float().mean()), 4)}
@@ -638,6 +658,8 @@ def main():
     ap.add_argument("--sweep-n", default=None, help="comma-separated sequence lengths (default: all)")
     ap.add_argument("--sweep-f", default=None, help="comma-separated diffuse-head fractions (default: all)")
     ap.add_argument("--sweep-alpha", default=None, help="comma-separated alpha values (default: 0.5,1,2)")
+    ap.add_argument("--graphs", action="store_true",
+                    help="sweep / compare: time each stage as a replayed CUDA graph (GPU time only)")
     ap.add_argument("--compare", default=None,
                     help="write the CRISP vs FlexPrefill latency comparison to this JSONL file")
     ap.add_argument("--compare-workloads", default="qwen_131k,llama_512k",

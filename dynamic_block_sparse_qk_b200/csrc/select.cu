@@ -343,6 +343,34 @@ __device__ void pe_find(const crisp_params& p, PeState* stp, uint32_t* gc, doubl
   for (int i = tid; i < nbk; i += 256) { gc[i] = 0; gs[i] = 0.0; }
 }
 
+// Adds this lane's entry (bucket bk, value s; take = false: no entry) to a
+// shared-memory histogram of counts and fp64 sums. The entries of a row are
+// close in value, so the lanes of a warp mostly hit one or two buckets:
+// lanes with the same bucket combine first (each lane links to the next lane
+// of its bucket, five pointer-jumping steps leave the group's sum in its
+// lowest lane) and only that lane updates shared memory. All 32 lanes call.
+__device__ inline void hist_add_warp(uint32_t* hc, double* hs, bool take, uint32_t bk, double s) {
+  const int lane = threadIdx.x & 31;
+  if (!__any_sync(0xffffffffu, take)) return;
+  const unsigned peers = __match_any_sync(0xffffffffu, bk);
+  const unsigned above = lane == 31 ? 0u : peers & (0xFFFFFFFFu << (lane + 1));
+  int nxt = above ? __ffs(above) - 1 : -1;
+#pragma unroll
+  for (int step = 0; step < 5; ++step) {
+    const int src = nxt >= 0 ? nxt : lane;
+    const double o = __shfl_sync(0xffffffffu, s, src);
+    const int on = __shfl_sync(0xffffffffu, nxt, src);
+    if (nxt >= 0) {
+      s += o;
+      nxt = on;
+    }
+  }
+  if (take && (peers & ((1u << lane) - 1u)) == 0u) {
+    atomicAdd(&hc[bk], uint32_t(__popc(peers)));
+    atomicAdd(&hs[bk], s);
+  }
+}
+
 __global__ void __launch_bounds__(256) pe_hist_kernel(crisp_params p, const int32_t* pattern,
                                                       void* ws, int level) {
   __shared__ uint32_t hc[4096];
@@ -362,11 +390,6 @@ __global__ void __launch_bounds__(256) pe_hist_kernel(crisp_params p, const int3
   const int rows_per = 8;
   const int q0 = blockIdx.x * rows_per, q1 = min(q0 + rows_per, nbv);
   const uint32_t hi_shift = shift + (level == 2 ? 8 : 12);
-  // The entries of a row are close in value, so the lanes of a warp mostly hit
-  // one or two buckets. Lanes with the same bucket combine first: each lane
-  // links to the next lane of its bucket, five pointer-jumping steps leave the
-  // group's sum in its lowest lane, and only that lane updates shared memory.
-  const int lane = threadIdx.x & 31;
   for (int qb = q0; qb < q1; ++qb) {
     const float* row = abar + size_t(qb) * nb;
     for (int c0 = 0; c0 <= qb; c0 += 256) {          // uniform trip count: the whole CTA iterates
@@ -383,24 +406,7 @@ __global__ void __launch_bounds__(256) pe_hist_kernel(crisp_params p, const int3
           s = double(v);
         }
       }
-      if (!__any_sync(0xffffffffu, take)) continue;
-      const unsigned peers = __match_any_sync(0xffffffffu, bk);
-      const unsigned above = lane == 31 ? 0u : peers & (0xFFFFFFFFu << (lane + 1));
-      int nxt = above ? __ffs(above) - 1 : -1;
-#pragma unroll
-      for (int step = 0; step < 5; ++step) {
-        const int src = nxt >= 0 ? nxt : lane;
-        const double o = __shfl_sync(0xffffffffu, s, src);
-        const int on = __shfl_sync(0xffffffffu, nxt, src);
-        if (nxt >= 0) {
-          s += o;
-          nxt = on;
-        }
-      }
-      if (take && (peers & ((1u << lane) - 1u)) == 0u) {
-        atomicAdd(&hc[bk], uint32_t(__popc(peers)));
-        atomicAdd(&hs[bk], s);
-      }
+      hist_add_warp(hc, hs, take, bk, s);
     }
   }
   __syncthreads();
@@ -471,6 +477,174 @@ __global__ void __launch_bounds__(256) pe_eqcount_kernel(crisp_params p, const i
     run += c;
   }
   if (tid == 0) *cnt = 0u;
+}
+
+// ---------------------------------------------------------------------------
+// The PE gamma cut of one head in one CTA, for triangles that fit in shared
+// memory (N_b(N_b+1)/2 <= kPeSmallMax, i.e. N_b <= 256: sequences up to 32k
+// tokens at block 128). It replaces the normalisation, the three histogram
+// launches and the tie count of the multi-kernel path with the same
+// arithmetic: rows normalised as in pe_normalize_kernel (written back for the
+// tile builder and kept in shared memory in flat order), the same three-level
+// radix select with fp64 bucket sums and the same cut search, and the same
+// per-row tie counts turned into an exclusive scan; it leaves the PeState and
+// eq_cnt that build_tiles_kernel reads. One CTA of 1024 threads per head.
+// ---------------------------------------------------------------------------
+constexpr int kPeSmallMax = 256 * 257 / 2;
+constexpr int kPeSmallThreads = 1024;
+constexpr size_t kPeSmallSmem = size_t(kPeSmallMax) * 4 + 4096 * 4 + 4096 * 8 + (kPeSmallThreads + 2) * 8 + 256 * 4;
+
+__global__ void __launch_bounds__(kPeSmallThreads) pe_small_cut_kernel(crisp_params p, const int32_t* pattern,
+                                                                      void* ws) {
+  extern __shared__ __align__(16) unsigned char sm_raw[];
+  double* hs = reinterpret_cast<double*>(sm_raw);                       // [4096]
+  double* scan = hs + 4096;                                             // [1024 + 2]
+  uint32_t* hc = reinterpret_cast<uint32_t*>(scan + kPeSmallThreads + 2);  // [4096]
+  uint32_t* rowc = hc + 4096;                                           // [256]
+  float* vals = reinterpret_cast<float*>(rowc + 256);                   // [kPeSmallMax]
+  __shared__ int ctl[2];
+  __shared__ PeState st;
+  const Workspace W = make_workspace(p);
+  const int nb = n_blocks(p);                               // stride
+  const int bh = blockIdx.x;
+  if (pattern[bh] != CRISP_PATTERN_PE) return;
+  const int nbv = (seq_len(p, bh / p.h_q) + p.block - 1) / p.block;   // this sequence's blocks
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int M = nbv * (nbv + 1) / 2;
+  float* abar = ws_ptr<float>(ws, W.abar) + size_t(bh) * nb * nb;
+  // (1) rows: combine the logits kernel's (max, sum) partials, normalise,
+  // divide by N_b (as pe_normalize_kernel), write back and keep in flat order
+  {
+    const int ntile = (nb + 63) / 64;
+    for (int qb = warp; qb < nbv; qb += kPeSmallThreads / 32) {
+      const int nt = qb / 64 + 1;
+      const float* pm = ws_ptr<float>(ws, W.stat_m) + (size_t(bh) * nb + qb) * ntile;
+      const float* ps = ws_ptr<float>(ws, W.stat_lo) + (size_t(bh) * nb + qb) * ntile;
+      float mx = -INFINITY;
+      for (int t = lane; t < nt; t += 32) mx = fmaxf(mx, pm[t]);
+      mx = warp_max(mx);
+      float sacc = 0.f;
+      for (int t = lane; t < nt; t += 32) sacc += ps[t] * exp2f(pm[t] - mx);
+      sacc = warp_sum(sacc);
+      const float inv = 1.0f / (sacc * float(nbv));
+      float* row = abar + size_t(qb) * nb;
+      float* vrow = vals + qb * (qb + 1) / 2;
+      for (int kb = lane; kb <= qb; kb += 32) {
+        const float v = exp2f(row[kb] - mx) * inv;
+        row[kb] = v;
+        vrow[kb] = v;
+      }
+    }
+  }
+  if (tid == 0) st = PeState{};
+  __syncthreads();
+  // (2) radix select of the cut value, three levels
+  const double g = double(p.gamma);
+  for (int level = 0; level < 3; ++level) {
+    int shift, nbk;
+    level_geom(level, shift, nbk);
+    for (int i = tid; i < nbk; i += kPeSmallThreads) { hc[i] = 0u; hs[i] = 0.0; }
+    __syncthreads();
+    const uint32_t hi_shift = shift + (level == 2 ? 8 : 12);
+    const uint32_t prefix = st.prefix;
+    for (int i0 = 0; i0 < M; i0 += kPeSmallThreads) {     // uniform trip count
+      const int i = i0 + tid;
+      bool take = false;
+      uint32_t bk = 0xFFFFFFFFu;
+      double sv = 0.0;
+      if (i < M) {
+        const float v = vals[i];
+        const uint32_t u = __float_as_uint(v);
+        if (level == 0 || (u >> hi_shift) == (prefix >> hi_shift)) {
+          take = true;
+          bk = (u >> shift) & uint32_t(nbk - 1);
+          sv = double(v);
+        }
+      }
+      hist_add_warp(hc, hs, take, bk, sv);
+    }
+    __syncthreads();
+    // the highest bucket whose descending cumulative sum reaches gamma:
+    // thread t owns the buckets counted from the top t*per .. t*per+per-1
+    const int per = nbk / kPeSmallThreads > 0 ? nbk / kPeSmallThreads : 1;
+    const int nact = nbk / per;
+    double own = 0.0;
+    if (tid < nact)
+      for (int i = 0; i < per; ++i) own += hs[nbk - 1 - (tid * per + i)];
+    scan[tid] = own;
+    if (tid == 0) { ctl[0] = -1; ctl[1] = 1 << 30; }
+    __syncthreads();
+    for (int bkt = tid; bkt < nbk; bkt += kPeSmallThreads)
+      if (hc[bkt]) atomicMin(&ctl[1], bkt);
+    for (int off = 1; off < kPeSmallThreads; off <<= 1) {
+      const double v = tid >= off ? scan[tid - off] : 0.0;
+      __syncthreads();
+      scan[tid] += v;
+      __syncthreads();
+    }
+    const double above0 = st.above_sum;
+    double run = above0 + (tid > 0 ? scan[tid - 1] : 0.0);
+    int cand = -1;
+    double cand_above = 0.0;
+    if (tid < nact) {
+      for (int i = 0; i < per; ++i) {
+        const int bkt = nbk - 1 - (tid * per + i);
+        const double v = hs[bkt];
+        if (run + v >= g) { cand = bkt; cand_above = run; atomicMax(&ctl[0], bkt); break; }
+        run += v;
+      }
+    }
+    __syncthreads();
+    if (cand >= 0 && cand == ctl[0]) scan[kPeSmallThreads] = cand_above;   // exactly one owner
+    __syncthreads();
+    if (tid == 0) {
+      PeState s2 = st;
+      const int best = ctl[0], lowest = ctl[1];
+      int cut = best;
+      if (cut < 0 && level > 0 && lowest < nbk) cut = lowest;   // rounding fell short: whole range
+      if (cut < 0) {
+        s2.all = 1;                                             // the whole triangle sums below gamma
+      } else {
+        const double above = cut == best ? scan[kPeSmallThreads] : above0 + scan[kPeSmallThreads - 1] - hs[cut];
+        s2.prefix |= uint32_t(cut) << shift;
+        s2.above_sum = above;
+        if (level == 2) {
+          const float tv = __uint_as_float(s2.prefix);
+          const double need = g - above;
+          double m = ceil(need / double(tv));
+          if (m < 1.0) m = 1.0;
+          const double cap = double(hc[cut]);
+          if (m > cap) m = cap;
+          s2.m_equal = uint32_t(m);
+        }
+      }
+      st = s2;
+    }
+    __syncthreads();
+    if (st.all) break;
+  }
+  // (3) per-row counts of entries equal to the cut value, exclusive scan
+  if (!st.all) {
+    const float tv = __uint_as_float(st.prefix);
+    for (int qb = warp; qb < nbv; qb += kPeSmallThreads / 32) {
+      const float* vrow = vals + qb * (qb + 1) / 2;
+      uint32_t c = 0;
+      for (int kb = lane; kb <= qb; kb += 32) c += vrow[kb] == tv;
+      c = __reduce_add_sync(0xffffffffu, c);
+      if (lane == 0) rowc[qb] = c;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t* ec = ws_ptr<uint32_t>(ws, W.eq_cnt) + size_t(bh) * nb;
+      uint32_t run = 0;
+      for (int qb = 0; qb < nbv; ++qb) {
+        const uint32_t c = rowc[qb];
+        ec[qb] = run;
+        run += c;
+      }
+    }
+  }
+  if (tid == 0) ws_ptr<PeState>(ws, W.pe_state)[bh] = st;
 }
 
 // ---------------------------------------------------------------------------
@@ -677,15 +851,23 @@ cudaError_t run_select(const crisp_params& p, const void* q, const void* k, cons
     if (p.head_dim == 64) pe_logits_kernel<64><<<grid, 256, 0, st>>>(p, pattern, ws);
     else pe_logits_kernel<128><<<grid, 256, 0, st>>>(p, pattern, ws);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (size_t(nb) * (nb + 1) / 2 <= size_t(kPeSmallMax)) {
+    // short sequences: normalisation, radix select and ties in one CTA per head
+    e = cudaFuncSetAttribute(pe_small_cut_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kPeSmallSmem));
+    if (e != cudaSuccess) return e;
+    pe_small_cut_kernel<<<BH, kPeSmallThreads, kPeSmallSmem, st>>>(p, pattern, ws);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  } else {
     pe_normalize_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, pattern, ws);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  for (int level = 0; level < 3; ++level) {
-    pe_hist_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, pattern, ws, level);
+    for (int level = 0; level < 3; ++level) {
+      pe_hist_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, pattern, ws, level);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    pe_eqcount_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, pattern, ws);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  pe_eqcount_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, pattern, ws);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   // (3) tile lists.
   build_tiles_kernel<<<dim3((nb + 7) / 8, BH), 256, 0, st>>>(p, pattern, ws, mask, tile_idx, tile_cnt);
   return cudaGetLastError();
