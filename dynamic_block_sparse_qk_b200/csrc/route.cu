@@ -91,9 +91,11 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
   __shared__ float part[RPP][D];
   const int R = p.block, nb = n_blocks(p);
   const int tid = threadIdx.x, c = tid % CPR, rg = tid / CPR;
-  // Grid-stride over (head, block): a head nobody needs is skipped once per
-  // CTA instead of launching a CTA per block of it.
-  for (int hy = 0; hy < nk + nq; ++hy) {
+  // Grid-stride over the flat (head, block) space: the blocks of the heads
+  // that are needed spread over all CTAs; a head nobody needs costs one check
+  // per item.
+  for (int item = blockIdx.x; item < (nk + nq) * nb; item += gridDim.x) {
+    const int hy = item / nb, kb = item % nb;
     const bool is_k = hy < nk;
     const int hh = is_k ? hy : hy - nk;
     if (pattern) {
@@ -111,7 +113,7 @@ __global__ void __launch_bounds__(256) pool_kernel(const __nv_bfloat16* __restri
     const int nbv = (len + R - 1) / R;
     const __nv_bfloat16* x = is_k ? k : q;
     float* out = is_k ? kbar : qbar;
-    for (int kb = blockIdx.x; kb < nbv; kb += gridDim.x) {
+    if (kb < nbv) {
       const int rows = min(R, len - kb * R);         // a partial last block averages what it holds
       const __nv_bfloat16* src = x + (size_t(hh) * p.seqlen + size_t(kb) * R) * D;
       float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -224,7 +226,7 @@ cudaError_t launch_pool(const crisp_params& p, const void* k, const void* q, int
                         const int32_t* pattern, float* kbar, float* qbar, cudaStream_t st) {
   if (nk + nq == 0) return cudaSuccess;
   const int nb = n_blocks(p);
-  const unsigned grid = unsigned(min(nb, 4 * 148));
+  const unsigned grid = unsigned(min((nk + nq) * nb, 4 * 148));
   const auto* kk = static_cast<const __nv_bfloat16*>(k);
   const auto* qq = static_cast<const __nv_bfloat16*>(q);
   if (p.head_dim == 64)

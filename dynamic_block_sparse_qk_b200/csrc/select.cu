@@ -162,13 +162,17 @@ __global__ void __launch_bounds__(256) pe_logits_kernel(crisp_params p, const in
   const Workspace W = make_workspace(p);
   const int nb = n_blocks(p);                               // stride
   const int BH = p.batch * p.h_q;
-  // Grid-stride over (PE head, lower-triangle 64x64 tile): heads that are
-  // not PE cost one check per CTA.
-  for (int bh = 0; bh < BH; ++bh) {
+  const int ntq_max = (nb + T - 1) / T, tiles_max = ntq_max * (ntq_max + 1) / 2;
+  // Grid-stride over the flat (head, lower-triangle 64x64 tile) space, so the
+  // tiles of all PE heads spread over the CTAs even when a head has only a
+  // few; a head that is not PE costs one check per item.
+  for (int item = blockIdx.x; item < BH * tiles_max; item += gridDim.x) {
+    const int bh = item / tiles_max, tt = item % tiles_max;
     if (pattern[bh] != CRISP_PATTERN_PE) continue;
     const int nbv = (seq_len(p, bh / p.h_q) + p.block - 1) / p.block;   // this sequence's blocks
     const int ntq = (nbv + T - 1) / T;
-    for (int tt = blockIdx.x; tt < ntq * (ntq + 1) / 2; tt += gridDim.x) {
+    if (tt >= ntq * (ntq + 1) / 2) continue;
+    {
       int tq = int((sqrtf(8.f * float(tt) + 1.f) - 1.f) * 0.5f);
       while ((tq + 1) * (tq + 2) / 2 <= tt) ++tq;
       while (tq * (tq + 1) / 2 > tt) --tq;

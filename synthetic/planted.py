@@ -82,6 +82,7 @@ WORKLOADS: Dict[str, Workload] = {
                      n_vertical=0, recency_peak=9.0, recency_freqs="rope"),
     "llama_32k": Workload("llama_32k", 1, 32, 8, 128, 32768, 128),
     "qwen_131k": Workload("qwen_131k", 1, 28, 4, 128, 131072, 128, sink_logit_range=(1.0, 6.0)),
+    "llama_8k": Workload("llama_8k", 1, 32, 8, 128, 8192, 128),
     "llama_128k": Workload("llama_128k", 1, 32, 8, 128, 131072, 128),
     "llama_512k": Workload("llama_512k", 1, 32, 8, 128, 524288, 128),
     # the same shapes with a decaying RoPE-style recency band (geometric

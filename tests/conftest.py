@@ -31,6 +31,8 @@ def pytest_terminal_summary(terminalreporter):
     tot = {"cases": len(reps), "heads": sum(r["heads"] for r in reps),
            "exempt_routes": sum(r["exempt_routes"] for r in reps),
            "exempt_blocks": sum(r["exempt_blocks"] for r in reps),
+           "exempt_differing": sum(r.get("exempt_differing", 0) for r in reps),
+           "routes_differing": sum(r.get("routes_differing", 0) for r in reps),
            "qblocks_compared": sum(r["qblocks_compared"] for r in reps),
            "attn_max_abs": max(r["attn_max_abs"] for r in reps)}
     terminalreporter.write_line("parity totals: " + json.dumps(tot, default=float))

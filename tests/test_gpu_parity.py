@@ -342,8 +342,10 @@ def test_llama_512k_alpha_schedule():
 
 
 # ---- sweep points beyond alpha = 1: selection in full, attention sampled
+# (at 512k only the mixed input: its 16 VS heads cover what the VS-only one
+# would, and the oracle's routing of 32 heads at 512k takes minutes)
 @pytest.mark.slow
-@pytest.mark.parametrize("seqlen,f", [(65536, 0.0), (65536, 0.5), (524288, 0.0), (524288, 0.5)])
+@pytest.mark.parametrize("seqlen,f", [(65536, 0.0), (65536, 0.5), (524288, 0.5)])
 def test_sweep_points_alpha_half_and_two(seqlen, f):
     w = sweep_workload(seqlen, f)
     nb = w.n_blocks
