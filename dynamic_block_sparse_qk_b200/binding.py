@@ -8,6 +8,7 @@ the library cannot be loaded, importing it raises.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 from typing import Optional
 
@@ -298,6 +299,14 @@ def crisp_prefill_host(p: CrispParams, q, k, v, o, ws, lse=None, seq_lens=None, 
     for t in (q, k, v, o, lse, seq_lens, pattern):
         if t is not None and (t.is_cuda or not t.is_contiguous()):
             raise ValueError("crisp_prefill_host takes contiguous host tensors")
+    n, d = p.seqlen, p.head_dim
+    want = {"q": (q, (p.batch, p.h_q, n, d), torch.bfloat16), "k": (k, (p.batch, p.h_kv, n, d), torch.bfloat16),
+            "v": (v, (p.batch, p.h_kv, n, d), torch.bfloat16), "o": (o, (p.batch, p.h_q, n, d), torch.bfloat16),
+            "lse": (lse, (p.batch, p.h_q, n), torch.float32), "seq_lens": (seq_lens, (p.batch,), torch.int32),
+            "pattern": (pattern, (p.batch * p.h_q,), torch.int32)}
+    for name, (t, shape, dtype) in want.items():
+        if t is not None and (t.dtype != dtype or t.numel() != math.prod(shape)):
+            raise ValueError(f"{name} must hold {math.prod(shape)} elements of {dtype}")
     _check("crisp_prefill_host", load_library().crisp_prefill_host(
         ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(seq_lens), _ptr(pattern),
         int(kv_per_chunk), _ptr(ws), ws.numel(), _stream(stream)))
