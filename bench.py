@@ -185,6 +185,22 @@ def stage_algorithmic_bytes(w, pattern, tiles: int) -> dict:
     return {"route": route, "select": select}
 
 
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# the sparse attention kernel, from an ncu capture of this bench's own
+# command on a B200 (1 pass; profiles/attn_tc_sparse_llama512k_dram.md).
+# Valid for the default hyper-parameters of the workload and the kernel as
+# captured; any other configuration reports null.
+ATTN_DRAM_BYTES = {"llama_512k": 156_760_839_168 + 4_371_607_040}
+
+
+def attn_traffic(w, args):
+    if (args.alpha, args.gamma, args.router, args.vs_rule, args.granularity) != (1.0, 0.95, "cstruct", "alpha", "tile"):
+        return None
+    if args.shard != "replicas" or w.lengths is not None:
+        return None
+    return ATTN_DRAM_BYTES.get(w.name)
+
+
 def executed_flops(tile_cnt_sum: int, block: int, d: int) -> float:
     """4 * B^2 * d per executed tile (QK^T and PV); diagonal tiles count in full."""
     return float(tile_cnt_sum) * 4.0 * block * block * d
@@ -352,7 +368,9 @@ def run_ours(args, rank, world, local_rank):
                      "frac_of_spec_2250": round(attn_tflops / 2250.0, 4),
                      "peak_source": f"{peaks['source']} bf16 "
                                     f"{'sustained' if peak == peaks['bf16_tflops_sustained'] else 'burst'}",
-                     "traffic": None},
+                     "traffic": attn_traffic(w_full, args),
+                     "traffic_unit": "bytes per launch (DRAM read + write, ncu)",
+                     "algorithmic_bytes": int(in_bytes + o.numel() * o.element_size() + lse.numel() * 4)},
         "stage_hbm": {k_: {"algorithmic_bytes": int(v_),
                            "achieved_gbs": round(v_ / (stages[k_] * 1e-3) / 1e9, 1),
                            "frac_of_hbm": round(v_ / (stages[k_] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
