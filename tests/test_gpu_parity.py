@@ -342,10 +342,11 @@ def test_llama_512k_alpha_schedule():
 
 
 # ---- sweep points beyond alpha = 1: selection in full, attention sampled
-# (at 512k only the mixed input: its 16 VS heads cover what the VS-only one
-# would, and the oracle's routing of 32 heads at 512k takes minutes)
+# (at 512k on the first, the last and one random query block per head: at
+# alpha = 0.5 every tile is selected and each sampled block costs the oracle
+# a full causal row)
 @pytest.mark.slow
-@pytest.mark.parametrize("seqlen,f", [(65536, 0.0), (65536, 0.5), (524288, 0.5)])
+@pytest.mark.parametrize("seqlen,f", [(65536, 0.0), (65536, 0.5), (524288, 0.0), (524288, 0.5)])
 def test_sweep_points_alpha_half_and_two(seqlen, f):
     w = sweep_workload(seqlen, f)
     nb = w.n_blocks
@@ -359,3 +360,14 @@ def test_llama_32k_rope_recency():
     w = WORKLOADS["llama_32k_rope"]
     reps = _check(w, qblocks_fn=lambda b, h: PU.sample_qblocks(w.n_blocks, 4, 7000 + h), expect_both=True)
     assert sum(r["pattern"] == O.VS for r in reps) == 24
+
+
+# ---- the FlexPrefill comparison path at scale (JSD routing, gamma-cumsum VS
+# index, Appendix A), as the latency comparison runs it
+@pytest.mark.slow
+@pytest.mark.parametrize("gamma", [0.95, 0.97])
+def test_flexprefill_path_llama_64k(gamma):
+    w = sweep_workload(65536, 0.25)
+    reps = _check(w, router="jsd", vs_rule="gamma", gamma=gamma, inputs=_device_inputs(w), keep_on_device=True,
+                  qblocks_fn=lambda b, h: PU.sample_qblocks(w.n_blocks, 4, 8000 + h))
+    assert {r["pattern"] for r in reps} == {O.VS, O.PE}
