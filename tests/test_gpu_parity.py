@@ -371,3 +371,15 @@ def test_flexprefill_path_llama_64k(gamma):
     reps = _check(w, router="jsd", vs_rule="gamma", gamma=gamma, inputs=_device_inputs(w), keep_on_device=True,
                   qblocks_fn=lambda b, h: PU.sample_qblocks(w.n_blocks, 4, 8000 + h))
     assert {r["pattern"] for r in reps} == {O.VS, O.PE}
+
+
+@pytest.mark.slow
+def test_llama_512k_rope_recency_sampled_heads():
+    # at 512k the RoPE far field pulls C_struct below tau_proxy, so every head
+    # takes the PE path; four heads (one per pair of KV groups), selection in
+    # full, attention on the first, the last and two random query blocks
+    w = WORKLOADS["llama_512k_rope"]
+    heads = (0, 9, 18, 27)
+    reps = _check(w, heads=heads, inputs=_device_inputs(w), keep_on_device=True,
+                  qblocks_fn=lambda b, h: PU.sample_qblocks(w.n_blocks, 2, 9000 + h))
+    assert len(reps) == len(heads)
