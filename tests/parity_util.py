@@ -153,20 +153,27 @@ def pe_exempt(a_bar: np.ndarray, gamma: float) -> np.ndarray:
 
 
 def oracle_for_alphas(q_head, k_head, oprms):
-    """Oracle results for parameter sets that differ only in alpha: routing
-    and the PE index (which alpha does not enter) once, then the VS index of
-    Algorithm 3 and its tile mask per alpha, with the same oracle functions
-    head_route_and_select composes."""
+    """Oracle results for parameter sets that differ only in their VS index
+    (alpha, or the alpha / median / gamma rule at one gamma and router):
+    routing and the PE index (which none of those enter) once, then the VS
+    index (Algorithm 3, or Algorithm 6 for the gamma rule) and its tile mask
+    per set, with the same oracle functions head_route_and_select composes."""
     base = O.head_route_and_select(q_head, k_head, oprms[0])
     outs = [base]
     n = q_head.shape[0]
+    p0 = oprms[0]
     for prm in oprms[1:]:
-        assert prm.vs_rule in ("alpha", "alpha_median") and prm.block == oprms[0].block
+        assert (prm.block, prm.gamma, prm.router, prm.tau_proxy, prm.tau_jsd, prm.granularity) == \
+            (p0.block, p0.gamma, p0.router, p0.tau_proxy, p0.tau_jsd, p0.granularity)
         r = dict(base)
         if base["pattern"] == O.VS:
-            floor = "median" if prm.vs_rule == "alpha_median" else "mean"
-            r["s_v"] = O.vs_index_alpha(base["p_v"], prm.alpha, prm.k_min_blocks, floor)
-            r["s_s"] = O.vs_index_alpha(base["p_s"], prm.alpha, prm.k_min_blocks, floor)
+            if prm.vs_rule == "gamma":
+                r["s_v"] = O.vs_index_gamma(base["p_v"], prm.gamma, prm.k_min_blocks)
+                r["s_s"] = O.vs_index_gamma(base["p_s"], prm.gamma, prm.k_min_blocks)
+            else:
+                floor = "median" if prm.vs_rule == "alpha_median" else "mean"
+                r["s_v"] = O.vs_index_alpha(base["p_v"], prm.alpha, prm.k_min_blocks, floor)
+                r["s_s"] = O.vs_index_alpha(base["p_s"], prm.alpha, prm.k_min_blocks, floor)
             r["mask"] = O.vs_tile_mask(r["s_v"], r["s_s"], O.n_blocks(n, prm.block), n, prm.block)
         outs.append(r)
     return outs

@@ -50,15 +50,17 @@ def _device_inputs(w):
     return out
 
 
-def _check_alphas(w, alphas, qblocks_fn, inputs, expect_both=False):
-    """One input, several alpha values: each alpha is a full GPU prefill
-    (route, select, attention) compared with the oracle; the oracle routes and
-    runs the PE index once per head and the VS index once per alpha."""
+def _check_alphas(w, alphas, qblocks_fn, inputs, expect_both=False, vs_rules=None):
+    """One input, several alpha values (or VS rules): each is a full GPU
+    prefill (route, select, attention) compared with the oracle; the oracle
+    routes and runs the PE index once per head and the VS index once per
+    setting."""
     q, k, v, _ = inputs
-    oprms = [PU.oracle_params(w, alpha=a) for a in alphas]
+    vs_rules = vs_rules or ["alpha"] * len(alphas)
+    oprms = [PU.oracle_params(w, alpha=a, vs_rule=r) for a, r in zip(alphas, vs_rules)]
     gpus = []
-    for a in alphas:
-        gpu = PU.run_gpu(w, q, k, v, alpha=a, keep_on_device=True)
+    for a, r in zip(alphas, vs_rules):
+        gpu = PU.run_gpu(w, q, k, v, alpha=a, vs_rule=r, keep_on_device=True)
         assert gpu["status"] == 0
         gpus.append(gpu)
     g = w.h_q // w.h_kv
@@ -74,7 +76,7 @@ def _check_alphas(w, alphas, qblocks_fn, inputs, expect_both=False):
             reps[i].append(PU.compare_head(gpus[i], 0, h, qh, kh, vh, w, oprms[i], qblocks_fn(i, h),
                                            orc=orcs[i]))
     for i, a in enumerate(alphas):
-        PU.record(f"{w.name} cstruct alpha alpha={a} gamma=0.95 tile", reps[i])
+        PU.record(f"{w.name} cstruct {vs_rules[i]} alpha={a} gamma=0.95 tile", reps[i])
         if expect_both:
             assert {r["pattern"] for r in reps[i]} == {O.VS, O.PE}
     return reps
@@ -325,9 +327,8 @@ def _sample32(nb, base):
 @pytest.mark.slow
 def test_qwen_131k_alpha_and_gamma():
     w = WORKLOADS["qwen_131k"]
-    inputs = _device_inputs(w)
-    for vs_rule in ("alpha", "gamma"):
-        _check(w, vs_rule=vs_rule, qblocks_fn=_sample32(w.n_blocks, 2000), inputs=inputs, keep_on_device=True)
+    _check_alphas(w, (1.0, 1.0), lambda i, h: PU.sample_qblocks(w.n_blocks, 30, 2000 + h), _device_inputs(w),
+                  vs_rules=["alpha", "gamma"])
 
 
 @pytest.mark.slow
