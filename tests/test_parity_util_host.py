@@ -11,9 +11,9 @@ import parity_util as PU
 from synthetic import WORKLOADS, make_qkv
 
 
-def _p_with_block_at_threshold(nb=20, alpha=1.0):
-    # sink 0.5, local 0.2, a flat background of 0.01 per middle block: the
-    # mean floor is (1 - 0.7) / 18 = 0.3 / 18; block 5 sits on alpha * mu
+def _p_with_blocks_at_threshold(nb=20):
+    # sink 0.5, local 0.2 and a flat background of 0.3 / 18 per middle block:
+    # the mean floor is (1 - 0.7) / 18, so every middle block sits on mu
     p = np.full(nb, 0.0)
     p[0], p[-1] = 0.5, 0.2
     p[1:-1] = 0.3 / (nb - 2)
@@ -21,7 +21,7 @@ def _p_with_block_at_threshold(nb=20, alpha=1.0):
 
 
 def test_vs_exempt_alpha_flags_blocks_on_the_threshold():
-    p = _p_with_block_at_threshold()
+    p = _p_with_blocks_at_threshold()
     mu = O.noise_floor(p)
     ex = PU.vs_exempt(p, "alpha", 1.0, 0.95, k_min=2)
     # every middle block equals mu exactly: all of them lie in the band; with
