@@ -522,7 +522,8 @@ def run_sweep(args, out_path):
             for line in f:
                 try:
                     d = json.loads(line)
-                    done.add((d["seq_len"], d["diffuse_frac"], d["alpha"], d.get("vs_rule", "alpha")))
+                    done.add((d["seq_len"], d["diffuse_frac"], d["alpha"], d.get("vs_rule", "alpha"),
+                              d.get("granularity", "tile")))
                 except (ValueError, KeyError):
                     pass
     dev = torch.device("cuda", 0)
@@ -533,7 +534,7 @@ def run_sweep(args, out_path):
     alphas = tuple(float(x) for x in args.sweep_alpha.split(",")) if args.sweep_alpha else SWEEP_ALPHA
     for n in ns:
         for f in fs:
-            todo = [a for a in alphas if (n, f, a, args.vs_rule) not in done]
+            todo = [a for a in alphas if (n, f, a, args.vs_rule, args.granularity) not in done]
             if not todo:
                 continue
             w = sweep_workload(n, f).with_(seed=args.seed)
@@ -544,10 +545,11 @@ def run_sweep(args, out_path):
             pj = C.params_for(q, k, block=w.block, router="jsd")
             pat_j = C.crisp_route(pj, q, k, ws)[0].clone()
             for a in todo:
-                p = C.params_for(q, k, block=w.block, alpha=a, vs_rule=args.vs_rule)
+                p = C.params_for(q, k, block=w.block, alpha=a, vs_rule=args.vs_rule, granularity=args.granularity)
                 pt = time_point(C, p, q, k, v, ws, timed, dev)
                 pat = pt.pop("_pattern")
-                rec = {"seq_len": n, "diffuse_frac": f, "alpha": a, "vs_rule": args.vs_rule, "workload": w.name,
+                rec = {"seq_len": n, "diffuse_frac": f, "alpha": a, "vs_rule": args.vs_rule, "granularity": args.granularity,
+                       "workload": w.name,
                        "timing": "cuda_graph" if args.graphs else "eager",
                        **pt, "dense_ms": round(dense_ms, 4),
                        "speedup_vs_dense": round(dense_ms / pt["total_ms"], 3),
